@@ -1,0 +1,60 @@
+// Internal host-side interface between the C-ABI layer (api.cu) and the
+// kernel files.  Launchers assume their arguments were validated by api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace bsq {
+
+// Count of kernels launched by the library (bsq_debug_launch_count).
+void note_launch();
+
+// Per-file flags of bounded waits that ran out (read and cleared with a
+// device synchronisation; used by tests only).
+uint32_t take_timeouts_gemm_w4a4();
+uint32_t take_timeouts_gemm_fp8();
+uint32_t take_timeouts_gemm_int8();
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// ---- launchers (quant.cu) ----
+cudaError_t launch_quant_nvfp4(const uint16_t *in, uint8_t *packed, uint8_t *scale, float scale2, int m, int k,
+                               cudaStream_t s);
+cudaError_t launch_quant_rowwise_fp8(const uint16_t *in, uint8_t *q, float *scale, int rows, int k,
+                                     cudaStream_t s);
+cudaError_t launch_quant_blockfp8(const uint16_t *in, uint8_t *q, float *scale, int n, int k, cudaStream_t s);
+cudaError_t launch_requant_blockfp8_to_rowwise(const uint8_t *w, const float *bscale, int n, int k, uint8_t *q,
+                                               float *scale, cudaStream_t s);
+cudaError_t launch_requant_w_nvfp4_int8(const uint8_t *packed, const uint8_t *sf, float scale2, int8_t *q,
+                                        float *scale, int n, int k, cudaStream_t s);
+cudaError_t launch_quant_act_int8_per32(const uint16_t *a, int8_t *q, float *scale, int m, int k,
+                                        cudaStream_t s);
+cudaError_t launch_amax_bf16(const uint16_t *x, size_t count, float *amax, cudaStream_t s);
+
+// ---- launchers (gemv_fp8.cu) ----
+cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *row_scale, uint16_t *out,
+                                     int m, int n, int k, cudaStream_t s);
+
+// ---- launchers (gemm_*.cu) ----
+cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
+                             const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k,
+                             cudaStream_t s);
+cudaError_t launch_fp8_gemm_rowscale(const uint8_t *a, const float *a_scale, const uint8_t *w,
+                                     const float *w_scale, uint16_t *out, int m, int n, int k, cudaStream_t s);
+cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const float *a_scale,
+                                         const float *w_scale, uint16_t *out, int m, int n, int k,
+                                         cudaStream_t s);
+
+// ---- tensor maps (tma.cu) ----
+// 2-D row-major tensor of `rows` x `cols` elements of `elem_bytes` bytes,
+// row stride `row_stride_bytes`; box of box_cols x box_rows.  swizzle128
+// selects the 128-byte swizzle (box_cols * elem_bytes must be 128 then).
+struct CUtensorMap_st_holder;
+bool make_tmap_2d(void *tmap_out, const void *base, int elem_bytes, uint64_t cols, uint64_t rows,
+                  uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128,
+                  bool elem_is_float);
+
+}  // namespace bsq

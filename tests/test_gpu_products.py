@@ -1,0 +1,248 @@
+"""GPU parity of the products (W4A4 GEMM, FP8 GEMV, FP8 GEMM, int8 per-32
+GEMM) against the CPU oracle on identical quantised codes:
+|gpu - oracle| <= 1e-2 |oracle| + 1e-3 sum|a*w|, element by element.  Sizes
+span several tiles with ragged edges; the full configurations run in the
+launch configuration the benchmark times, checked on sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+import int8_gemm_gemv_b200 as bsq
+import oracle
+from int8_gemm_gemv_b200 import synth
+from gpu_helpers import bf16_out, check_tol, empty, host, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _no_timeouts():
+    yield
+    assert bsq.debug_take_timeouts() == 0
+
+
+def sample_rows(m, count=16, seed=0):
+    g = np.random.default_rng(seed)
+    r = set([0, m - 1, min(m - 1, 127), min(m - 1, 128)])
+    r.update(g.integers(0, m, count).tolist())
+    return np.array(sorted(r), np.int64)
+
+
+# ------------------------------------------------------------------ W4A4 ---
+
+def nvfp4_from_oracle(m, n, k, seed, heavy=True):
+    a_bf, w_bf = synth.w4a4_inputs(m, n, k, seed=seed, heavy_tailed=heavy)
+    sb2 = float(np.float32(oracle.amax_bf16(w_bf)) / np.float32(6 * 448))
+    ap, asf = oracle.quant_nvfp4(a_bf, 1.0)
+    wp, wsf = oracle.quant_nvfp4(w_bf, sb2)
+    return ap, asf, wp, wsf, 1.0, sb2
+
+
+def nvfp4_random(m, n, k, seed):
+    ap = synth.uniform_bytes((m, k // 2), seed, 11)
+    wp = synth.uniform_bytes((n, k // 2), seed, 12)
+    asf = synth.uniform_bytes((m, k // 16), seed, 13, 0x20, 0x60)
+    wsf = synth.uniform_bytes((n, k // 16), seed, 14, 0x20, 0x60)
+    return ap, asf, wp, wsf, 1.0, 2.0**-7
+
+
+def run_w4a4(ap, asf, wp, wsf, sa2, sb2):
+    m, n, k = ap.shape[0], wp.shape[0], ap.shape[1] * 2
+    out = bf16_out((m, n))
+    bsq.w4a4_gemm(to_dev(ap), to_dev(asf), to_dev(wp), to_dev(wsf), out, sa2, sb2, m, n, k)
+    torch.cuda.synchronize()
+    return host(out, np.uint16)
+
+
+@pytest.mark.parametrize("mnk", [(16, 256, 512), (200, 300, 512), (129, 520, 768), (1, 8, 256)])
+def test_w4a4_small_and_ragged(mnk):
+    m, n, k = mnk
+    args = nvfp4_from_oracle(m, n, k, seed=1)
+    g = run_w4a4(*args)
+    ob, _, ab = oracle.w4a4_gemm(*args)
+    check_tol(g, ob, ab, f"w4a4 {mnk}")
+
+
+def test_w4a4_structured_one_hot():
+    """One-hot activation rows pick single weight elements: checks nibble
+    order, scale placement per row and per 16-block, and the M/N tiling."""
+    m, n, k = 256, 512, 512
+    g = np.random.default_rng(5)
+    a = np.zeros((m, k), np.uint8)
+    cols = g.integers(0, k, m)
+    a[np.arange(m), cols] = 2  # 1.0
+    ap = (a[:, 0::2] | (a[:, 1::2] << 4)).astype(np.uint8)
+    asf = synth.uniform_bytes((m, k // 16), 5, 1, 0x30, 0x48)
+    wp = synth.uniform_bytes((n, k // 2), 5, 2)
+    wsf = synth.uniform_bytes((n, k // 16), 5, 3, 0x30, 0x48)
+    got = run_w4a4(ap, asf, wp, wsf, 1.0, 1.0)
+    ob, ex, ab = oracle.w4a4_gemm(ap, asf, wp, wsf, 1.0, 1.0)
+    check_tol(got, ob, ab, "w4a4 one-hot")
+    # each product is exact in FP32 and BF16 keeps 8 bits: exact match
+    # whenever the exact value is BF16-representable
+    exact_rep = oracle.bf16_to_f32(ob).astype(np.float64) == ex
+    assert np.array_equal(got[exact_rep], ob[exact_rep])
+
+
+def test_w4a4_realistic_mid():
+    args = nvfp4_from_oracle(512, 2048, 5120, seed=0)
+    g = run_w4a4(*args)
+    rows = sample_rows(512, 24)
+    ob, _, ab = oracle.w4a4_gemm(*args, rows=rows)
+    check_tol(g[rows], ob, ab, "w4a4 512x2048x5120")
+
+
+@pytest.mark.parametrize("m", [4096, 512])
+def test_w4a4_full_size(m):
+    n, k = 17408, 5120
+    args = nvfp4_random(m, n, k, seed=2)
+    g = run_w4a4(*args)
+    rows = sample_rows(m, 12)
+    ob, _, ab = oracle.w4a4_gemm(*args, rows=rows)
+    check_tol(g[rows], ob, ab, f"w4a4 {m}x{n}x{k}")
+
+
+# ------------------------------------------------------------------ GEMV ---
+
+def run_gemv(inp, wq, ws):
+    m, k = inp.shape
+    n = wq.shape[0]
+    out = bf16_out((m, n))
+    bsq.fp8_gemv_rowscale(to_dev(inp), to_dev(wq), to_dev(ws), out, m, n, k)
+    torch.cuda.synchronize()
+    return host(out, np.uint16)
+
+
+@pytest.fixture(scope="module")
+def gemv_weight():
+    _, w_bf = synth.gemv_inputs(1, 5120, 5120, seed=0)
+    return oracle.quant_rowwise_fp8(w_bf)
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 8, 9, 16])
+def test_gemv_cfg2(gemv_weight, m):
+    wq, ws = gemv_weight
+    inp = synth.normal_bf16((m, 5120), 1.0, 0, 3)
+    g = run_gemv(inp, wq, ws)
+    ob, _, ab = oracle.fp8_gemv_rowscale(inp, wq, ws)
+    check_tol(g, ob, ab, f"gemv m={m}")
+
+
+def test_gemv_row_independent_of_batch(gemv_weight):
+    """A row computed alone, or in a batch of 2, 8 or 16, gives the same bits
+    (fp8_gemv_batch.rs: the batched kernels are bit-identical per row)."""
+    wq, ws = gemv_weight
+    inp = synth.normal_bf16((16, 5120), 1.0, 1, 3)
+    full = run_gemv(inp, wq, ws)
+    for m in (1, 2, 8, 15):
+        part = run_gemv(inp[:m].copy(), wq, ws)
+        assert np.array_equal(part, full[:m]), m
+
+
+@pytest.mark.parametrize("nk", [(1000, 1040), (17, 16), (4095, 64)])
+def test_gemv_ragged(nk):
+    n, k = nk
+    inp, w_bf = synth.gemv_inputs(16, n, k, seed=2)
+    wq, ws = oracle.quant_rowwise_fp8(w_bf)
+    for m in (1, 5, 16):
+        g = run_gemv(inp[:m].copy(), wq, ws)
+        ob, _, ab = oracle.fp8_gemv_rowscale(inp[:m], wq, ws)
+        check_tol(g, ob, ab, f"gemv {m}x{n}x{k}")
+
+
+def test_gemv_lm_head_shape():
+    n, k = 151936, 5120
+    wq = synth.uniform_bytes((n, k), 0, 21, 0, 0x7F) | (synth.uniform_bytes((n, k), 0, 22, 0, 2) << 7)
+    ws = synth.uniform_f32((n,), 0, 23, 1e-4, 1e-3)
+    inp = synth.normal_bf16((2, k), 1.0, 0, 24)
+    g = run_gemv(inp, wq, ws)
+    cols = sample_rows(n, 200, seed=3)
+    ob, _, ab = oracle.fp8_gemv_rowscale(inp, wq[cols], ws[cols])
+    check_tol(g[:, cols], ob, ab, "gemv lm_head")
+
+
+# -------------------------------------------------------------- FP8 GEMM ---
+
+def run_fp8_gemm(a, sa, w, sw):
+    m, k = a.shape
+    n = w.shape[0]
+    out = bf16_out((m, n))
+    bsq.fp8_gemm_rowscale(to_dev(a), to_dev(sa), to_dev(w), to_dev(sw), out, m, n, k)
+    torch.cuda.synchronize()
+    return host(out, np.uint16)
+
+
+@pytest.mark.parametrize("mnk", [(23, 256, 256), (300, 520, 1040), (128, 256, 128)])
+def test_fp8_gemm_small_and_ragged(mnk):
+    m, n, k = mnk
+    a_bf, w_bf = synth.blockfp8_inputs(m, n, k, seed=1)
+    a, sa = oracle.quant_rowwise_fp8(a_bf)
+    w, sw = oracle.quant_rowwise_fp8(w_bf)
+    g = run_fp8_gemm(a, sa, w, sw)
+    ob, _, ab = oracle.fp8_gemm_rowscale(a, sa, w, sw)
+    check_tol(g, ob, ab, f"fp8 gemm {mnk}")
+
+
+def test_fp8_gemm_full_size():
+    m, n, k = 8192, 10240, 5120
+    a = synth.uniform_bytes((m, k), 0, 31, 0, 0x7F) | (synth.uniform_bytes((m, k), 0, 32, 0, 2) << 7)
+    w = synth.uniform_bytes((n, k), 0, 33, 0, 0x7F) | (synth.uniform_bytes((n, k), 0, 34, 0, 2) << 7)
+    sa = synth.uniform_f32((m,), 0, 35, 1e-3, 1e-2)
+    sw = synth.uniform_f32((n,), 0, 36, 1e-5, 1e-4)
+    g = run_fp8_gemm(a, sa, w, sw)
+    rows = sample_rows(m, 12)
+    ob, _, ab = oracle.fp8_gemm_rowscale(a, sa, w, sw, rows=rows)
+    check_tol(g[rows], ob, ab, "fp8 gemm 8192x10240x5120")
+
+
+# -------------------------------------------------------------- int8 GEMM --
+
+def run_int8(a, w, sa, sw):
+    m, k = a.shape
+    n = w.shape[0]
+    out = bf16_out((m, n))
+    bsq.int8_blockscaled_gemm(to_dev(a), to_dev(w), to_dev(sa), to_dev(sw), out, m, n, k)
+    torch.cuda.synchronize()
+    return host(out, np.uint16)
+
+
+@pytest.mark.parametrize("mnk", [(64, 128, 128), (200, 300, 640), (129, 136, 1024)])
+def test_int8_small_and_ragged(mnk):
+    m, n, k = mnk
+    a_bf, w_bf = synth.w4a8_inputs(m, n, k, seed=1)
+    s2 = float(np.float32(oracle.amax_bf16(w_bf)) / np.float32(6 * 448))
+    wp, wsf = oracle.quant_nvfp4(w_bf, s2)
+    w, sw = oracle.requant_w_nvfp4_int8(wp, wsf, s2)
+    a, sa = oracle.quant_act_int8_per32(a_bf)
+    g = run_int8(a, w, sa, sw)
+    ob, _, ab = oracle.int8_blockscaled_gemm(a, w, sa, sw)
+    check_tol(g, ob, ab, f"int8 {mnk}")
+
+
+def test_int8_prefill_two_launches():
+    m, n, k = 96, 256, 512
+    a_bf, w_bf = synth.w4a8_inputs(m, n, k, seed=3)
+    w = synth.uniform_int8((n, k), 3, 40)
+    sw = synth.uniform_f32((n, k // 32), 3, 41, 1e-4, 1e-3)
+    out = bf16_out((m, n))
+    a_i8, a_s = empty((m, k), torch.int8), empty((m, k // 32), torch.float32)
+    n0 = bsq.debug_launch_count()
+    bsq.int8_w4a8_prefill(to_dev(a_bf), to_dev(w), to_dev(sw), a_i8, a_s, out, m, n, k)
+    assert bsq.debug_launch_count() == n0 + 2
+    torch.cuda.synchronize()
+    a, sa = oracle.quant_act_int8_per32(a_bf)
+    assert np.array_equal(host(a_i8), a) and np.array_equal(host(a_s), sa)
+    ob, _, ab = oracle.int8_blockscaled_gemm(a, w, sa, sw)
+    check_tol(host(out, np.uint16), ob, ab, "int8 prefill")
+
+
+def test_int8_full_size():
+    m, n, k = 2048, 5120, 17408
+    a = synth.uniform_int8((m, k), 0, 42)
+    w = synth.uniform_int8((n, k), 0, 43)
+    sa = synth.uniform_f32((m, k // 32), 0, 44, 1e-3, 1e-1)
+    sw = synth.uniform_f32((n, k // 32), 0, 45, 1e-5, 1e-4)
+    g = run_int8(a, w, sa, sw)
+    rows = sample_rows(m, 10)
+    ob, _, ab = oracle.int8_blockscaled_gemm(a, w, sa, sw, rows=rows)
+    check_tol(g[rows], ob, ab, "int8 2048x5120x17408")
