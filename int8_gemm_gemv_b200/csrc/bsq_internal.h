@@ -16,6 +16,7 @@ void note_launch();
 uint32_t take_timeouts_gemm_w4a4();
 uint32_t take_timeouts_gemm_fp8();
 uint32_t take_timeouts_gemm_int8();
+uint32_t take_timeouts_gemv();
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
@@ -56,5 +57,11 @@ struct CUtensorMap_st_holder;
 bool make_tmap_2d(void *tmap_out, const void *base, int elem_bytes, uint64_t cols, uint64_t rows,
                   uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128,
                   bool elem_is_float);
+
+// 3-D view of a row-major [rows, k_bytes] byte matrix as (128 B, rows,
+// k_bytes/128 chunks) so one TMA copy moves box_rows x (box_chunks * 128 B)
+// with the 128-byte swizzle.  Needs k_bytes % 128 == 0.
+bool make_tmap_rows_chunks(void *tmap_out, const void *base, uint64_t k_bytes, uint64_t rows, uint32_t box_rows,
+                           uint32_t box_chunks);
 
 }  // namespace bsq

@@ -3,20 +3,23 @@
 //   C[m, n] = scaleA2 * scaleB2 * sum_k e2m1(A) e4m3(sfA) e2m1(W) e4m3(sfW)
 //
 // Design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: A [128 x 256 elem], W [256 x 256 elem] (packed,
-//               128-byte swizzle) and the two raw scale tiles per K block,
-//               into a 4-stage ring guarded by mbarriers.
-//   warp 2      scale-factor re-layout: the scale tiles arrive row-major
-//               ([rows, 16 bytes] per 256-wide K block); the MMA reads its
-//               scales from tensor memory in 32-lane groups where lane i of
-//               column j holds row 32j+i.  This warp rewrites each stage's
-//               scale bytes in shared memory into that order (in place).
-//   warp 1      MMA issuer (one thread): copies the stage's scales into
-//               tensor memory (tcgen05.cp, replicated to the four lane
-//               groups) and issues four 128x256x64 block-scaled MMAs per
-//               K block into one FP32 accumulator in tensor memory.
-//   warps 4..7  epilogue: tensor memory -> registers -> scale -> BF16 ->
-//               global, one 32-lane quarter of the tile each.
+//   warp 0       TMA producer: A [128 x 256 elem], W [256 x 256 elem] (packed,
+//                128-byte swizzle) and the two raw scale tiles per K block,
+//                into a 4-stage ring guarded by mbarriers.
+//   warps 12..15 scale-factor writers: the scale tiles arrive row-major
+//                ([rows, 16 bytes] per 256-wide K block); the MMA reads its
+//                scales from tensor memory where, in every 32-lane group,
+//                lane i of column j holds row 32j+i.  Each writer warp reads
+//                the stage's scales from shared memory and stores them with
+//                tcgen05.st into its own lane group (the layout is replicated
+//                in all four groups).  Doing this with plain tensor-memory
+//                stores keeps it off the tensor core's instruction queue, so
+//                it overlaps the MMAs.
+//   warp 1       MMA issuer (one thread): four 128x256x64 block-scaled MMAs
+//                per K block into one FP32 accumulator in tensor memory.
+//   warps 4..11  epilogue: tensor memory -> registers -> scale -> BF16 ->
+//                global; warp w owns lane group w % 4 and column half
+//                (w - 4) / 4 of the tile.
 // Tiles go M-fastest, so consecutive CTAs share the same weight panel (the
 // `w4a4_gemm_mfast` raster) and the whole working set stays in L2.
 //
@@ -40,7 +43,7 @@ constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0;                  // 256 FP32 columns
 constexpr int SF_COL = 256;                 // per stage: 16 (A) + 32 (B)
 constexpr int SF_STAGE_COLS = 48;
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 
 static __device__ unsigned int g_timeouts;
 
@@ -77,11 +80,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
             mbar_init(&S->full[s], 1);
-            mbar_init(&S->sfready[s], 1);
+            mbar_init(&S->sfready[s], 4);
             mbar_init(&S->empty[s], 1);
         }
         mbar_init(&S->tfull, 1);
-        mbar_init(&S->tempty, 4);
+        mbar_init(&S->tempty, 8);
         mbar_init(&S->drain, 1);
         S->abort = 0;
         fence_mbar_init();
@@ -127,8 +130,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (uint32_t i = first; i < it; i++) mbar_wait(&S->full[i % STAGES], (i / STAGES) & 1, &g_timeouts);
             }
         }
-    } else if (warp == 2) {
-        // ------------------------------------- scale-factor re-layout
+    } else if (warp >= 12) {
+        // ------------------------------------------ scale-factor writers
+        const int q = warp & 3;
+        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         uint32_t it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -139,30 +144,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                // raw: row r at r*16, word j = scales of MMA step j.
-                // atom (step j, group g): word 4*i + q = raw word (128g + 32q + i, j).
-                uint4 *sa = reinterpret_cast<uint4 *>(sfa_tile(s));
-                uint4 *sb = reinterpret_cast<uint4 *>(sfb_tile(s));
-                uint4 ra[4], rb[2][4];
+                // raw tile: row r at r*16 bytes, word j = the 4 scales of MMA step j
+                const uint4 *sa = reinterpret_cast<const uint4 *>(sfa_tile(s));
+                const uint4 *sb = reinterpret_cast<const uint4 *>(sfb_tile(s));
+                uint4 va[4], vb[8];
 #pragma unroll
-                for (int q = 0; q < 4; q++) ra[q] = sa[32 * q + lane];
+                for (int j = 0; j < 4; j++) va[j] = sa[32 * j + lane];
 #pragma unroll
-                for (int g = 0; g < 2; g++)
+                for (int j = 0; j < 8; j++) vb[j] = sb[32 * j + lane];
+                // column (step * groups + j) of this lane = row 32j + lane, step
+                uint32_t ra[16], rb[32];
 #pragma unroll
-                    for (int q = 0; q < 4; q++) rb[g][q] = sb[128 * g + 32 * q + lane];
-                __syncwarp();
-                sa[0 * 32 + lane] = make_uint4(ra[0].x, ra[1].x, ra[2].x, ra[3].x);
-                sa[1 * 32 + lane] = make_uint4(ra[0].y, ra[1].y, ra[2].y, ra[3].y);
-                sa[2 * 32 + lane] = make_uint4(ra[0].z, ra[1].z, ra[2].z, ra[3].z);
-                sa[3 * 32 + lane] = make_uint4(ra[0].w, ra[1].w, ra[2].w, ra[3].w);
-#pragma unroll
-                for (int g = 0; g < 2; g++) {
-                    sb[(0 * 2 + g) * 32 + lane] = make_uint4(rb[g][0].x, rb[g][1].x, rb[g][2].x, rb[g][3].x);
-                    sb[(1 * 2 + g) * 32 + lane] = make_uint4(rb[g][0].y, rb[g][1].y, rb[g][2].y, rb[g][3].y);
-                    sb[(2 * 2 + g) * 32 + lane] = make_uint4(rb[g][0].z, rb[g][1].z, rb[g][2].z, rb[g][3].z);
-                    sb[(3 * 2 + g) * 32 + lane] = make_uint4(rb[g][0].w, rb[g][1].w, rb[g][2].w, rb[g][3].w);
+                for (int j = 0; j < 4; j++) {
+                    ra[0 + j] = va[j].x;
+                    ra[4 + j] = va[j].y;
+                    ra[8 + j] = va[j].z;
+                    ra[12 + j] = va[j].w;
                 }
-                fence_proxy_async_smem();
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    rb[0 + j] = vb[j].x;
+                    rb[8 + j] = vb[j].y;
+                    rb[16 + j] = vb[j].z;
+                    rb[24 + j] = vb[j].w;
+                }
+                const uint32_t col = tmem + lane_off + SF_COL + s * SF_STAGE_COLS;
+                tmem_st_32x32b_x16(col, ra);
+                tmem_st_32x32b_x32(col + 16, rb);
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S->sfready[s]);
             }
@@ -183,20 +193,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < nkb; kb++, it++) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(&S->sfready[s], ph, &g_timeouts) || aborted(S)) {
+                    if (!mbar_wait(&S->full[s], ph, &g_timeouts) || !mbar_wait(&S->sfready[s], ph, &g_timeouts) ||
+                        aborted(S)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t sfa_col = tmem + SF_COL + s * SF_STAGE_COLS;
                     const uint32_t sfb_col = sfa_col + 16;
-                    const uint32_t sa = smem_u32(sfa_tile(s)), sb = smem_u32(sfb_tile(s));
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        tmem_cp_32x128b_warpx4(sfa_col + 4 * j, sdesc_rows16(sa + j * 512));
-                        tmem_cp_32x128b_warpx4(sfb_col + 8 * j, sdesc_rows16(sb + (2 * j) * 512));
-                        tmem_cp_32x128b_warpx4(sfb_col + 8 * j + 4, sdesc_rows16(sb + (2 * j + 1) * 512));
-                    }
                     const uint32_t a0 = smem_u32(a_tile(s)), b0 = smem_u32(b_tile(s));
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4) {
         // ----------------------------------------------------- epilogue
-        const int q = warp - 4;
+        const int q = warp & 3, h = (warp - 4) >> 2;
         uint32_t tc = 0;
         const bool vec_ok = (N % 8) == 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tc++) {
@@ -228,11 +232,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int row = mt * BM + 32 * q + lane;
             uint16_t *orow = out + (int64_t)row * N;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; c++) {
+            for (int cc = 0; cc < BN / 64; cc++) {
+                const int c = h * (BN / 64) + cc;  // 32-column chunk of the tile
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem + ACC_COL + ((uint32_t)(32 * q) << 16) + c * 32, r);
                 tmem_ld_wait();
-                if (c == BN / 32 - 1) {
+                if (cc == BN / 64 - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S->tempty);

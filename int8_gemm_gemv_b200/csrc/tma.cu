@@ -42,6 +42,23 @@ bool make_tmap_2d(void *tmap_out, const void *base, int elem_bytes, uint64_t col
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_rows_chunks(void *tmap_out, const void *base, uint64_t k_bytes, uint64_t rows, uint32_t box_rows,
+                           uint32_t box_chunks) {
+    // dims (innermost first): 128 bytes of a chunk, rows (stride k_bytes),
+    // 128-byte chunks along K (stride 128); one box = box_rows x box_chunks
+    // chunks, landing as [chunk][row][128 B] with the 128-byte swizzle.
+    auto fn = encode_fn();
+    if (!fn || k_bytes % 128) return false;
+    const cuuint64_t dims[3] = {128, rows, k_bytes / 128};
+    const cuuint64_t strides[2] = {k_bytes, 128};
+    const cuuint32_t box[3] = {128, box_rows, box_chunks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(reinterpret_cast<CUtensorMap *>(tmap_out), CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int sm_count() {
     static int cached[64] = {};
     int dev = 0;
