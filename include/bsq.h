@@ -204,6 +204,35 @@ BSQ_API bsq_status int8_w4a8_prefill(const uint16_t *a_bf16, const int8_t *w_i8,
                              int m, int n, int k, bsq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * int8_w4a8_prefill_noalloc -- the same two launches as int8_w4a8_prefill,
+ * for callers that cannot allocate device memory and therefore cannot pass
+ * the two scratch buffers: code whose device memory is all owned by another
+ * allocator (a framework's caching allocator, a fixed arena handed out by the
+ * host application), plug-ins that have no allocation API at hand, and
+ * latency-critical paths that must not call cudaMalloc, which may
+ * synchronise the device.  No counterpart on the pages: their launcher
+ * always takes caller-owned scratch.
+ *   a_bf16 BF16 [m, k]; w_i8 int8 [n, k]; w_scale FP32 [n, k/32]; out BF16
+ *   [m, n]; all 16-byte aligned.  Result identical to int8_w4a8_prefill.
+ * Scratch: one fixed array inside the library, 45 MiB, room for m * k <=
+ * 41,943,040 activation elements.  Every GPU on which the library's device
+ * code is loaded reserves it until the process exits.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.
+ * This entry point allocates nothing and calls no allocating routine.
+ * All calls share the array and it keeps the last call's contents; each
+ * call writes every scratch byte it reads, so nothing needs clearing, but
+ * two calls whose executions overlap on the GPU (different streams, or
+ * different host threads) race on it and must be serialised by the caller.
+ * Errors: those of int8_w4a8_prefill; m * k above the limit ->
+ * BSQ_ERR_UNSUPPORTED (nothing launched); the address lookup failing ->
+ * BSQ_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+BSQ_API bsq_status int8_w4a8_prefill_noalloc(const uint16_t *a_bf16, const int8_t *w_i8,
+                                             const float *w_scale, uint16_t *out,
+                                             int m, int n, int k, bsq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * requant_blockfp8_to_rowwise -- dispatch_proj_rowwise.rs,
  * `rowwise_pair_passthrough` and `requant_weight_rowwise_fp8_cached`.
  *   tag == BSQ_FP8_PER_ROW: *w_used = w, *scale_used = scale; nothing is

@@ -18,7 +18,7 @@ __all__ = [
     "BSQ_ERR_CUDA", "BSQ_FP8_PER_ROW", "BSQ_FP8_BLOCK_SCALED", "BSQ_FP8_SINGLE_SCALE", "BSQ_BF16",
     "BSQ_NVFP4", "quantize_bf16_to_nvfp4", "w4a4_gemm", "fp8_gemv_rowscale", "quant_rowwise_fp8",
     "quant_blockfp8", "requant_w_nvfp4_int8", "quant_act_int8_per32", "int8_blockscaled_gemm",
-    "int8_w4a8_prefill", "requant_blockfp8_to_rowwise", "fp8_gemm_rowscale", "bsq_amax_bf16",
+    "int8_w4a8_prefill", "int8_w4a8_prefill_noalloc", "requant_blockfp8_to_rowwise", "fp8_gemm_rowscale", "bsq_amax_bf16",
     "status_string", "debug_launch_count", "debug_take_timeouts", "library_path", "lib",
 ]
 
@@ -53,6 +53,7 @@ _SIGS = {
     "quant_act_int8_per32": [_P, _P, _P, _I, _I, _P],
     "int8_blockscaled_gemm": [_P, _P, _P, _P, _P, _I, _I, _I, _P],
     "int8_w4a8_prefill": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P],
+    "int8_w4a8_prefill_noalloc": [_P, _P, _P, _P, _I, _I, _I, _P],
     "requant_blockfp8_to_rowwise": [_I, _P, _P, _I, _I, _P, _P, ctypes.POINTER(_P), ctypes.POINTER(_P), _P],
     "fp8_gemm_rowscale": [_P, _P, _P, _P, _P, _I, _I, _I, _P],
     "bsq_amax_bf16": [_P, ctypes.c_size_t, _P, _P],
@@ -159,6 +160,13 @@ def int8_blockscaled_gemm(a_i8, w_i8, a_scale, w_scale, out, m, n, k, stream=Non
 def int8_w4a8_prefill(a_bf16, w_i8, w_scale, a_i8_scratch, a_scale_scratch, out, m, n, k, stream=None):
     _call("int8_w4a8_prefill", _ptr(a_bf16), _ptr(w_i8), _ptr(w_scale), _ptr(a_i8_scratch),
           _ptr(a_scale_scratch), _ptr(out), m, n, k, _stream(stream))
+
+
+def int8_w4a8_prefill_noalloc(a_bf16, w_i8, w_scale, out, m, n, k, stream=None):
+    """int8_w4a8_prefill with the activation scratch inside the library (for
+    callers that cannot allocate device memory); see include/bsq.h."""
+    _call("int8_w4a8_prefill_noalloc", _ptr(a_bf16), _ptr(w_i8), _ptr(w_scale), _ptr(out), m, n, k,
+          _stream(stream))
 
 
 def requant_blockfp8_to_rowwise(tag, w, scale, n, k, w_out, scale_out, stream=None):
