@@ -2,101 +2,133 @@
 // (gemm_fp4.rs, `w4a4_gemm` and `w4a4_gemm_mfast`):
 //   C[m, n] = scaleA2 * scaleB2 * sum_k e2m1(A) e4m3(sfA) e2m1(W) e4m3(sfW)
 //
-// Design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0       TMA producer: A [128 x 256 elem], W [256 x 256 elem] (packed,
-//                128-byte swizzle) and the two raw scale tiles per K block,
-//                into a 4-stage ring guarded by mbarriers.
-//   warps 12..15 scale-factor writers: the scale tiles arrive row-major
-//                ([rows, 16 bytes] per 256-wide K block); the MMA reads its
-//                scales from tensor memory where, in every 32-lane group,
-//                lane i of column j holds row 32j+i.  Each writer warp reads
-//                the stage's scales from shared memory and stores them with
-//                tcgen05.st into its own lane group (the layout is replicated
-//                in all four groups).  Doing this with plain tensor-memory
-//                stores keeps it off the tensor core's instruction queue, so
-//                it overlaps the MMAs.
-//   warp 1       MMA issuer (one thread): four 128x256x64 block-scaled MMAs
-//                per K block into one FP32 accumulator in tensor memory.
-//   warps 4..11  epilogue: tensor memory -> registers -> scale -> BF16 ->
-//                global; warp w owns lane group w % 4 and column half
-//                (w - 4) / 4 of the tile.
-// Tiles go M-fastest, so consecutive CTAs share the same weight panel (the
-// `w4a4_gemm_mfast` raster) and the whole working set stays in L2.
+// Design: CTA pairs (clusters of two SMs), persistent over 256 x 256 output
+// tiles.  One pair MMA (tcgen05.mma.cta_group::2, 256 x 256 x 64) runs on
+// both SMs' tensor cores: each CTA holds 128 rows of A and 128 of the 256
+// weight rows in its shared memory and receives 128 x 256 of the output in
+// its tensor memory.  Each SM therefore loads half the weight tile a 1-SM
+// 128 x 256 tile would need, which is what lets the FP4 tensor cores be
+// fed from L2.
+//
+// Per CTA (512 threads):
+//   warp 0        TMA producer.  A and weight halves go into a 4-stage ring;
+//                 their arrival is counted on the even CTA's barrier (the
+//                 MMA issuer's).  The raw scale tiles (A: own 128 rows, W:
+//                 all 256 rows) arrive on a local barrier.
+//   warps 12..15  scale-factor writers: the scale tiles arrive row-major
+//                 ([rows, 16 bytes] per 256-wide K block); the MMA reads its
+//                 scales from tensor memory where, in every 32-lane group,
+//                 lane i of column j holds row 32j+i.  They write that layout
+//                 with tcgen05.st (off the tensor core's queue) and tell the
+//                 even CTA.
+//   warp 1        tensor-memory allocation for the pair; in the even CTA,
+//                 lane 0 issues the pair MMAs and commits them to both CTAs.
+//   warps 4..11   epilogue: tensor memory -> registers -> scale -> BF16 ->
+//                 swizzled shared-memory staging -> TMA store; warp w owns
+//                 lane group w % 4 and column half (w - 4) / 4 of the CTA's
+//                 128 x 256 block, and releases tensor memory as soon as its
+//                 part is in registers.
+// Tiles go M-fastest, so consecutive pairs share the same weight panel (the
+// `w4a4_gemm_mfast` raster) and the working set stays in L2.  No load uses
+// cluster multicast.
 //
 // Every mbarrier wait is bounded; on a timeout the kernel records it, stops
 // issuing work, drains what it issued, frees tensor memory and exits.
+#include <cstring>
+
 #include "bsq_common.cuh"
 
 namespace bsq {
 
 namespace {
 
-constexpr int BM = 128, BN = 256;
-constexpr int BK_BYTES = 128;  // 256 FP4 elements
+constexpr int BM = 128;                  // rows of A per CTA (256 per pair)
+constexpr int BN = 256;                  // output columns per tile
+constexpr int BNH = BN / 2;              // weight rows per CTA
+constexpr int BK_BYTES = 128;            // 256 FP4 elements
 constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK_BYTES;      // 16 KB
-constexpr int B_BYTES = BN * BK_BYTES;      // 32 KB
-constexpr int SFA_BYTES = BM * 16;          // 2 KB
-constexpr int SFB_BYTES = BN * 16;          // 4 KB
+constexpr int A_BYTES = BM * BK_BYTES;   // 16 KB
+constexpr int B_BYTES = BNH * BK_BYTES;  // 16 KB
+constexpr int SFA_BYTES = BM * 16;       // 2 KB
+constexpr int SFB_BYTES = BN * 16;       // 4 KB (all 256 weight rows)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int TMEM_COLS = 512;
-constexpr int ACC_COL = 0;                  // 256 FP32 columns
-constexpr int SF_COL = 256;                 // per stage: 16 (A) + 32 (B)
+constexpr int ACC_COL = 0;               // 256 FP32 columns
+constexpr int SF_COL = 256;              // per stage: 16 (A) + 32 (W)
 constexpr int SF_STAGE_COLS = 48;
 constexpr int kThreads = 512;
+constexpr int kEpiWarps = 8, kSfWarps = 4;
+// output staging: per epilogue warp 32 rows x 128 columns of BF16, as two
+// TMA store boxes of 32 rows x 64 columns (128-byte rows, 128-byte swizzle)
+constexpr int OUT_BOX_COLS = 64, OUT_BOX_ROWS = 32;
+constexpr int OUT_BOX_BYTES = OUT_BOX_COLS * 2 * OUT_BOX_ROWS;  // 4 KB
+constexpr int OUT_WARP_BYTES = 2 * OUT_BOX_BYTES;
+constexpr int OUT_BYTES = kEpiWarps * OUT_WARP_BYTES;             // 64 KB
+
+static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned");
+static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
 
 static __device__ unsigned int g_timeouts;
 
 struct Smem {
-    uint64_t full[STAGES];
-    uint64_t sfready[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t ab_full[STAGES];  // even CTA: A + W halves of both CTAs landed
+    uint64_t sf_full[STAGES];  // local: raw scale tiles landed
+    uint64_t sfready[STAGES];  // even CTA: both CTAs' scales are in tensor memory
+    uint64_t empty[STAGES];    // local: the pair MMAs of this stage are done
     uint64_t tfull, tempty, drain;
     uint32_t tmem_base;
     uint32_t abort;
 };
 
-constexpr size_t kSmemBytes = 1024 /* alignment slack */ + (size_t)STAGES * STAGE_BYTES + sizeof(Smem);
+constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + OUT_BYTES + sizeof(Smem);
 
 __device__ __forceinline__ bool aborted(volatile Smem *s) { return s->abort != 0; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     k_w4a4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                uint16_t *__restrict__ out, float scale_ab, int M, int N, int K) {
+                const __grid_constant__ CUtensorMap tmOut, int use_tma_store, uint16_t *__restrict__ out,
+                float scale_ab, int M, int N, int K) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Smem *S = reinterpret_cast<Smem *>(base + (size_t)STAGES * STAGE_BYTES);
+    uint8_t *out_stage = base + (size_t)STAGES * STAGE_BYTES;
+    Smem *S = reinterpret_cast<Smem *>(out_stage + OUT_BYTES);
     auto a_tile = [&](int s) { return base + (size_t)s * STAGE_BYTES; };
     auto b_tile = [&](int s) { return base + (size_t)s * STAGE_BYTES + A_BYTES; };
     auto sfa_tile = [&](int s) { return base + (size_t)s * STAGE_BYTES + A_BYTES + B_BYTES; };
     auto sfb_tile = [&](int s) { return base + (size_t)s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
+    const uint32_t rank = cluster_ctarank();  // 0: issues the pair MMAs
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int tiles_m = (M + 2 * BM - 1) / (2 * BM), tiles_n = (N + BN - 1) / BN;
     const int num_tiles = tiles_m * tiles_n;
     const int nkb = K / 256;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
-            mbar_init(&S->full[s], 1);
-            mbar_init(&S->sfready[s], 4);
+            mbar_init(&S->ab_full[s], 1);
+            mbar_init(&S->sf_full[s], 1);
+            mbar_init(&S->sfready[s], 2 * kSfWarps);
             mbar_init(&S->empty[s], 1);
         }
         mbar_init(&S->tfull, 1);
-        mbar_init(&S->tempty, 8);
+        mbar_init(&S->tempty, 2 * kEpiWarps);
         mbar_init(&S->drain, 1);
         S->abort = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&S->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(&S->tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
+    // cluster addresses of the even CTA's barriers
+    auto leader = [&](uint64_t *bar) { return mapa_shared(smem_u32(bar), 0); };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -107,8 +139,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tmSFB);
             uint32_t it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            for (int t = pair; t < num_tiles && ok; t += npairs) {
                 const int mt = t % tiles_m, nt = t / tiles_m;
+                const int arow = mt * 2 * BM + (int)rank * BM, brow = nt * BN + (int)rank * BNH;
                 for (int kb = 0; kb < nkb; kb++, it++) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
@@ -116,31 +149,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&S->full[s], STAGE_BYTES);
-                    tma_load_2d(a_tile(s), &tmA, &S->full[s], kb * BK_BYTES, mt * BM);
-                    tma_load_2d(b_tile(s), &tmB, &S->full[s], kb * BK_BYTES, nt * BN);
-                    tma_load_2d(sfa_tile(s), &tmSFA, &S->full[s], kb * 16, mt * BM);
-                    tma_load_2d(sfb_tile(s), &tmSFB, &S->full[s], kb * 16, nt * BN);
+                    if (rank == 0) mbar_arrive_expect_tx(&S->ab_full[s], 2 * (A_BYTES + B_BYTES));
+                    const uint32_t abar = leader(&S->ab_full[s]);
+                    tma_load_2d_pair(a_tile(s), &tmA, abar, kb * BK_BYTES, arow);
+                    tma_load_2d_pair(b_tile(s), &tmB, abar, kb * BK_BYTES, brow);
+                    mbar_arrive_expect_tx(&S->sf_full[s], SFA_BYTES + SFB_BYTES);
+                    tma_load_2d(sfa_tile(s), &tmSFA, &S->sf_full[s], kb * 16, arow);
+                    tma_load_2d(sfb_tile(s), &tmSFB, &S->sf_full[s], kb * 16, nt * BN);
                 }
             }
             if (!ok) {
                 S->abort = 1;
-                // let the copies already issued land before the CTA can exit
+                // let this CTA's scale copies land before it can exit
                 const uint32_t first = it > STAGES ? it - STAGES : 0;
-                for (uint32_t i = first; i < it; i++) mbar_wait(&S->full[i % STAGES], (i / STAGES) & 1, &g_timeouts);
+                for (uint32_t i = first; i < it; i++)
+                    mbar_wait(&S->sf_full[i % STAGES], (i / STAGES) & 1, &g_timeouts);
             }
         }
-    } else if (warp >= 12) {
+    } else if (warp >= 4 + kEpiWarps) {
         // ------------------------------------------ scale-factor writers
         const int q = warp & 3;
         const uint32_t lane_off = (uint32_t)(32 * q) << 16;
         uint32_t it = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int t = pair; t < num_tiles && ok; t += npairs) {
             for (int kb = 0; kb < nkb; kb++, it++) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
-                if (!mbar_wait(&S->full[s], ph, &g_timeouts) || aborted(S)) {
+                if (!mbar_wait(&S->sf_full[s], ph, &g_timeouts) || aborted(S)) {
                     ok = false;
                     break;
                 }
@@ -174,18 +210,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&S->sfready[s]);
+                if (lane == 0) mbar_arrive_cluster(leader(&S->sfready[s]));
             }
         }
         if (!ok && lane == 0) S->abort = 1;
     } else if (warp == 1) {
-        // --------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = idesc_nvf4(BM, BN);
+        // ---------------------------------------- pair MMA issuer (even CTA)
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = idesc_nvf4(2 * BM, BN);
             uint32_t it = 0, tc = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, tc++) {
-                if (!mbar_wait(&S->tempty, (tc & 1) ^ 1, &g_timeouts) || aborted(S)) {
+            for (int t = pair; t < num_tiles && ok; t += npairs, tc++) {
+                if (!mbar_wait_cluster(&S->tempty, (tc & 1) ^ 1, &g_timeouts) || aborted(S)) {
                     ok = false;
                     break;
                 }
@@ -193,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < nkb; kb++, it++) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(&S->full[s], ph, &g_timeouts) || !mbar_wait(&S->sfready[s], ph, &g_timeouts) ||
-                        aborted(S)) {
+                    if (!mbar_wait(&S->ab_full[s], ph, &g_timeouts) ||
+                        !mbar_wait_cluster(&S->sfready[s], ph, &g_timeouts) || aborted(S)) {
                         ok = false;
                         break;
                     }
@@ -204,69 +240,104 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t a0 = smem_u32(a_tile(s)), b0 = smem_u32(b_tile(s));
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
-                        mma_nvf4(tmem + ACC_COL, sdesc_k_sw128(a0 + 32 * j), sdesc_k_sw128(b0 + 32 * j), idesc,
-                                 sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
+                        mma_nvf4_pair(tmem + ACC_COL, sdesc_k_sw128(a0 + 32 * j), sdesc_k_sw128(b0 + 32 * j), idesc,
+                                      sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
                     }
-                    tc_commit(&S->empty[s]);
+                    tc_commit_pair_multicast(&S->empty[s], 0x3);
                 }
                 if (!ok) break;
-                tc_commit(&S->tfull);
+                tc_commit_pair_multicast(&S->tfull, 0x3);
             }
             if (!ok) S->abort = 1;
             // wait for every tensor-core operation this thread issued
-            tc_commit(&S->drain);
+            tc_commit_pair_multicast(&S->drain, 0x1);
             mbar_wait(&S->drain, 0, &g_timeouts);
         }
     } else if (warp >= 4) {
         // ----------------------------------------------------- epilogue
+        // Drain the whole accumulator block into registers (packed BF16)
+        // before releasing tensor memory, so the next tile's MMAs never wait
+        // behind this tile's global stores; then write through shared memory
+        // with TMA stores (coalesced, asynchronous).
         const int q = warp & 3, h = (warp - 4) >> 2;
+        uint8_t *stage = out_stage + (warp - 4) * OUT_WARP_BYTES;
         uint32_t tc = 0;
-        const bool vec_ok = (N % 8) == 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, tc++) {
+        const uint32_t tempty_leader = leader(&S->tempty);
+        if (lane == 0) prefetch_tensormap(&tmOut);
+        for (int t = pair; t < num_tiles; t += npairs, tc++) {
             const int mt = t % tiles_m, nt = t / tiles_m;
             if (!mbar_wait(&S->tfull, tc & 1, &g_timeouts) || aborted(S)) {
                 if (lane == 0) S->abort = 1;
                 break;
             }
             tc_fence_after();
-            const int row = mt * BM + 32 * q + lane;
-            uint16_t *orow = out + (int64_t)row * N;
-#pragma unroll 1
-            for (int cc = 0; cc < BN / 64; cc++) {
-                const int c = h * (BN / 64) + cc;  // 32-column chunk of the tile
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ACC_COL + ((uint32_t)(32 * q) << 16) + c * 32, r);
+            const uint32_t tbase = tmem + ACC_COL + ((uint32_t)(32 * q) << 16) + h * 128;
+            uint32_t pk[64];  // 128 columns of this lane's row as BF16 pairs
+#pragma unroll
+            for (int half = 0; half < 2; half++) {
+                uint32_t r0[32], r1[32];
+                tmem_ld_32x32b_x32(tbase + half * 64, r0);
+                tmem_ld_32x32b_x32(tbase + half * 64 + 32, r1);
                 tmem_ld_wait();
-                if (cc == BN / 64 - 1) {
+                if (half == 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&S->tempty);
+                    if (lane == 0) mbar_arrive_cluster(tempty_leader);
                 }
-                if (row >= M) continue;
-                const int n0 = nt * BN + c * 32;
-                if (vec_ok && n0 + 32 <= N) {
-                    uint32_t p[16];
 #pragma unroll
-                    for (int i = 0; i < 16; i++)
-                        p[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * scale_ab, __uint_as_float(r[2 * i + 1]) * scale_ab);
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + n0);
+                for (int i = 0; i < 16; i++) {
+                    pk[half * 32 + i] = pack_bf16x2(__uint_as_float(r0[2 * i]) * scale_ab,
+                                                    __uint_as_float(r0[2 * i + 1]) * scale_ab);
+                    pk[half * 32 + 16 + i] = pack_bf16x2(__uint_as_float(r1[2 * i]) * scale_ab,
+                                                         __uint_as_float(r1[2 * i + 1]) * scale_ab);
+                }
+            }
+            const int row0 = mt * 2 * BM + (int)rank * BM + 32 * q;  // first row of this warp
+            const int col0 = nt * BN + h * 128;
+            if (use_tma_store) {
+                // the previous tile's stores must have finished reading the staging buffer
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+                // box b holds columns [64b, 64b+64) of the warp's 32 x 128 block;
+                // lane = row; 16-byte unit u of a row sits at u ^ (row & 7)
 #pragma unroll
-                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
-                } else {
+                for (int bx = 0; bx < 2; bx++)
 #pragma unroll
-                    for (int i = 0; i < 32; i++)
-                        if (n0 + i < N)
-                            orow[n0 + i] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(r[i]) * scale_ab));
+                    for (int u = 0; u < 8; u++) {
+                        const uint32_t off = bx * OUT_BOX_BYTES + lane * 128 + ((u ^ (lane & 7)) << 4);
+                        *reinterpret_cast<uint4 *>(stage + off) =
+                            make_uint4(pk[bx * 32 + 4 * u], pk[bx * 32 + 4 * u + 1], pk[bx * 32 + 4 * u + 2],
+                                       pk[bx * 32 + 4 * u + 3]);
+                    }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && row0 < M) {  // boxes past the last row or column are skipped
+                    if (col0 < N) tma_store_2d(&tmOut, stage, col0, row0);
+                    if (col0 + OUT_BOX_COLS < N) tma_store_2d(&tmOut, stage + OUT_BOX_BYTES, col0 + OUT_BOX_COLS, row0);
+                    bulk_commit_group();
+                }
+            } else {
+                const int row = row0 + lane;
+                if (row < M) {
+                    uint16_t *orow = out + (int64_t)row * N;
+#pragma unroll
+                    for (int i = 0; i < 64; i++) {
+                        const int n = col0 + 2 * i;
+                        if (n < N) orow[n] = (uint16_t)(pk[i] & 0xFFFF);
+                        if (n + 1 < N) orow[n + 1] = (uint16_t)(pk[i] >> 16);
+                    }
                 }
             }
         }
+        if (lane == 0) bulk_wait_group0();  // stores complete before the CTA exits
     }
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();  // no pair MMA or cross-CTA signal is in flight after this
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc_pair(tmem, TMEM_COLS);
     }
 }
 
@@ -279,13 +350,32 @@ uint32_t take_timeouts_gemm_w4a4() {
     return v;
 }
 
+// CTA pairs that can be resident at once (cached per device).
+static int w4a4_max_pairs(cudaLaunchConfig_t cfg) {
+    static int cached[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    cfg.gridDim = dim3(sm_count());
+    if (cudaOccupancyMaxActiveClusters(&n, k_w4a4_gemm, &cfg) != cudaSuccess || n <= 0) n = sm_count() / 2;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
+    return n;
+}
+
 cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
                              const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k,
                              cudaStream_t s) {
     alignas(64) CUtensorMap tA, tB, tSA, tSB;
     const uint64_t kb = (uint64_t)k / 2, ks = (uint64_t)k / 16;
+    // TMA stores need 16-byte output rows (n % 8 == 0); otherwise plain stores
+    alignas(64) CUtensorMap tO;
+    const int use_tma_store = (n % 8) == 0;
+    if (use_tma_store && !make_tmap_2d(&tO, out, 2, n, m, (uint64_t)n * 2, OUT_BOX_COLS, OUT_BOX_ROWS, true, false))
+        return cudaErrorInvalidValue;
+    if (!use_tma_store) memset(&tO, 0, sizeof(tO));
     if (!make_tmap_2d(&tA, a_packed, 1, kb, m, kb, BK_BYTES, BM, true, false) ||
-        !make_tmap_2d(&tB, w_packed, 1, kb, n, kb, BK_BYTES, BN, true, false) ||
+        !make_tmap_2d(&tB, w_packed, 1, kb, n, kb, BK_BYTES, BNH, true, false) ||
         !make_tmap_2d(&tSA, a_scale, 1, ks, m, ks, 16, BM, false, false) ||
         !make_tmap_2d(&tSB, w_scale, 1, ks, n, ks, 16, BN, false, false))
         return cudaErrorInvalidValue;
@@ -297,11 +387,24 @@ cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, co
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    const int tiles = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
-    const int grid = tiles < sm_count() ? tiles : sm_count();
-    k_w4a4_gemm<<<grid, kThreads, kSmemBytes, s>>>(tA, tB, tSA, tSB, out, scale_ab, m, n, k);
+    const int tiles = ((m + 2 * BM - 1) / (2 * BM)) * ((n + BN - 1) / BN);
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int max_pairs = w4a4_max_pairs(cfg);
+    const int pairs = tiles < max_pairs ? tiles : max_pairs;
+    cfg.gridDim = dim3(2 * pairs);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_w4a4_gemm, tA, tB, tSA, tSB, tO, use_tma_store, out, scale_ab, m, n, k);
     note_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace bsq

@@ -20,8 +20,10 @@
 // The summation order of one output never depends on M.
 //
 // Launched with programmatic stream serialization: the prologue overlaps the
-// previous kernel on the stream, and every global-memory access waits for it
-// (griddepcontrol.wait), so the ordering of the stream is unchanged.
+// previous kernel on the stream -- including an L2 prefetch of the CTA's
+// first 256 KB of weight rows, which is safe before the dependency because
+// L2 is the GPU's point of coherence -- and every load and store waits for
+// it (griddepcontrol.wait), so the ordering of the stream is unchanged.
 //
 // Inside a 64-byte K chunk, lane (g = lane/4, t = lane%4) reads bytes
 // [16t, 16t+16) of tile rows g and g+8 and the same K range of activation
@@ -33,13 +35,19 @@ namespace bsq {
 
 namespace {
 
-constexpr int kConsumers = 16;
+#ifndef BSQ_GEMV_CONSUMERS
+#define BSQ_GEMV_CONSUMERS 16
+#define BSQ_GEMV_KS 1024
+#define BSQ_GEMV_STAGES 6
+#endif
+constexpr int kConsumers = BSQ_GEMV_CONSUMERS;
 constexpr int kThreads = 32 * (kConsumers + 1);
-constexpr int KS = 1024;                     // K bytes per stage
+constexpr int KS = BSQ_GEMV_KS;              // K bytes per stage (64 per consumer warp)
 constexpr int TILE_BYTES = 16 * KS;          // 16 KB: 16 rows x 1024 B
 constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // two tiles
-constexpr int STAGES = 6;                    // 192 KB ring
+constexpr int STAGES = BSQ_GEMV_STAGES;      // ring of STAGES x 2 tiles
 constexpr int BOX = 128;                     // TMA box: 128 B x 16 rows
+constexpr uint64_t kPrefetchBytes = 256 << 10;  // per CTA, before the stream dependency
 
 static __device__ unsigned int g_timeouts;
 
@@ -102,7 +110,7 @@ __device__ __forceinline__ uint32_t stage_offset(int u, int w, int r, int t) {
 
 template <int MT>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_fp8_gemv(const __grid_constant__ CUtensorMap tmW, const uint16_t *__restrict__ X,
+    k_fp8_gemv(const __grid_constant__ CUtensorMap tmW, const uint8_t *__restrict__ wptr, const uint16_t *__restrict__ X,
                const float *__restrict__ row_scale, uint16_t *__restrict__ out, int M, int N, int K, int tm3d) {
     extern __shared__ uint8_t smem_raw[];
     // the next kernel of the stream may start its own prologue now
@@ -125,9 +133,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         S->abort = 0;
         fence_mbar_init();
     }
+    // Start pulling this CTA's first weight rows into L2 while the previous
+    // kernel of the stream may still be running (up to kPrefetchBytes; a
+    // tile of 16 rows is one contiguous block of 16*K bytes).
+    if (threadIdx.x == 0) {
+        const uint8_t *wbase = reinterpret_cast<const uint8_t *>(wptr);
+        uint64_t done = 0;
+        for (int t = t_begin; t < t_end && done < kPrefetchBytes; t++) {
+            const int rows = min(16, N - 16 * t);
+            const uint64_t bytes = (uint64_t)rows * K;
+            prefetch_l2_bulk(wbase + (uint64_t)t * 16 * K, (uint32_t)bytes);
+            done += bytes;
+        }
+    }
     __syncthreads();
-    // everything above touched shared memory only; global memory waits for
-    // the previous kernel of the stream
+    // everything above touched shared memory or only prefetched into L2;
+    // global memory is read and written after the previous kernel of the
+    // stream has completed
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == kConsumers) {
@@ -275,8 +297,8 @@ uint32_t take_timeouts_gemv() {
 }
 
 template <int MT>
-static cudaError_t launch_mt(const CUtensorMap &tm, int tm3d, const uint16_t *in, const float *row_scale,
-                             uint16_t *out, int m, int n, int k, cudaStream_t s) {
+static cudaError_t launch_mt(const CUtensorMap &tm, int tm3d, const uint8_t *w, const uint16_t *in,
+                             const float *row_scale, uint16_t *out, int m, int n, int k, cudaStream_t s) {
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -298,7 +320,7 @@ static cudaError_t launch_mt(const CUtensorMap &tm, int tm3d, const uint16_t *in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_fp8_gemv<MT>, tm, in, row_scale, out, m, n, k, tm3d);
+    return cudaLaunchKernelEx(&cfg, k_fp8_gemv<MT>, tm, w, in, row_scale, out, m, n, k, tm3d);
 }
 
 cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *row_scale, uint16_t *out,
@@ -310,8 +332,8 @@ cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const
     const bool ok = tm3d ? make_tmap_rows_chunks(&tm, w, k, n, 16, KS / BOX)
                          : make_tmap_2d(&tm, w, 1, k, n, k, BOX, 16, true, false);
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = m <= 8 ? launch_mt<1>(tm, tm3d, in, row_scale, out, m, n, k, s)
-                           : launch_mt<2>(tm, tm3d, in, row_scale, out, m, n, k, s);
+    cudaError_t e = m <= 8 ? launch_mt<1>(tm, tm3d, w, in, row_scale, out, m, n, k, s)
+                           : launch_mt<2>(tm, tm3d, w, in, row_scale, out, m, n, k, s);
     note_launch();
     return e;
 }
