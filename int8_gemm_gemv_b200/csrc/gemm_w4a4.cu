@@ -11,7 +11,7 @@
 // fed from L2.
 //
 // Per CTA (512 threads):
-//   warp 0        TMA producer.  A and weight halves go into a 4-stage ring;
+//   warp 0        TMA producer.  A and weight halves go into a 5-stage ring;
 //                 their arrival is counted on the even CTA's barrier (the
 //                 MMA issuer's).  The raw scale tiles (A: own 128 rows, W:
 //                 all 256 rows) arrive on a local barrier.
@@ -46,7 +46,7 @@ constexpr int BM = 128;                  // rows of A per CTA (256 per pair)
 constexpr int BN = 256;                  // output columns per tile
 constexpr int BNH = BN / 2;              // weight rows per CTA
 constexpr int BK_BYTES = 128;            // 256 FP4 elements
-constexpr int STAGES = 4;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BK_BYTES;   // 16 KB
 constexpr int B_BYTES = BNH * BK_BYTES;  // 16 KB
 constexpr int SFA_BYTES = BM * 16;       // 2 KB
@@ -58,12 +58,12 @@ constexpr int SF_COL = 256;              // per stage: 16 (A) + 32 (W)
 constexpr int SF_STAGE_COLS = 48;
 constexpr int kThreads = 512;
 constexpr int kEpiWarps = 8, kSfWarps = 4;
-// output staging: per epilogue warp 32 rows x 128 columns of BF16, as two
-// TMA store boxes of 32 rows x 64 columns (128-byte rows, 128-byte swizzle)
+// output staging: per epilogue warp one TMA store box of 32 rows x 64
+// columns of BF16 (128-byte rows, 128-byte swizzle), used twice per tile
 constexpr int OUT_BOX_COLS = 64, OUT_BOX_ROWS = 32;
 constexpr int OUT_BOX_BYTES = OUT_BOX_COLS * 2 * OUT_BOX_ROWS;  // 4 KB
-constexpr int OUT_WARP_BYTES = 2 * OUT_BOX_BYTES;
-constexpr int OUT_BYTES = kEpiWarps * OUT_WARP_BYTES;             // 64 KB
+constexpr int OUT_WARP_BYTES = OUT_BOX_BYTES;
+constexpr int OUT_BYTES = kEpiWarps * OUT_WARP_BYTES;             // 32 KB
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned");
 static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
@@ -295,26 +295,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int row0 = mt * 2 * BM + (int)rank * BM + 32 * q;  // first row of this warp
             const int col0 = nt * BN + h * 128;
             if (use_tma_store) {
-                // the previous tile's stores must have finished reading the staging buffer
-                if (lane == 0) bulk_wait_group_read0();
-                __syncwarp();
-                // box b holds columns [64b, 64b+64) of the warp's 32 x 128 block;
-                // lane = row; 16-byte unit u of a row sits at u ^ (row & 7)
+                // box bx holds columns [64bx, 64bx+64) of the warp's 32 x 128
+                // block; lane = row; 16-byte unit u of a row sits at u ^ (row & 7)
 #pragma unroll
-                for (int bx = 0; bx < 2; bx++)
+                for (int bx = 0; bx < 2; bx++) {
+                    // the previous store must have finished reading the box
+                    if (lane == 0) bulk_wait_group_read0();
+                    __syncwarp();
 #pragma unroll
                     for (int u = 0; u < 8; u++) {
-                        const uint32_t off = bx * OUT_BOX_BYTES + lane * 128 + ((u ^ (lane & 7)) << 4);
+                        const uint32_t off = lane * 128 + ((u ^ (lane & 7)) << 4);
                         *reinterpret_cast<uint4 *>(stage + off) =
                             make_uint4(pk[bx * 32 + 4 * u], pk[bx * 32 + 4 * u + 1], pk[bx * 32 + 4 * u + 2],
                                        pk[bx * 32 + 4 * u + 3]);
                     }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0 && row0 < M) {  // boxes past the last row or column are skipped
-                    if (col0 < N) tma_store_2d(&tmOut, stage, col0, row0);
-                    if (col0 + OUT_BOX_COLS < N) tma_store_2d(&tmOut, stage + OUT_BOX_BYTES, col0 + OUT_BOX_COLS, row0);
-                    bulk_commit_group();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    // boxes past the last row or column are skipped
+                    if (lane == 0 && row0 < M && col0 + bx * OUT_BOX_COLS < N) {
+                        tma_store_2d(&tmOut, stage, col0 + bx * OUT_BOX_COLS, row0);
+                        bulk_commit_group();
+                    }
                 }
             } else {
                 const int row = row0 + lane;
