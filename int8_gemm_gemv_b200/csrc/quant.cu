@@ -12,7 +12,10 @@
 //   BF16 -> int8    gemm_dense_int8.rs, `int8_gemm_faith2_prefill` step (a)
 //
 // Every pinned FP32 step uses an explicit round-to-nearest intrinsic so the
-// compiler cannot contract or reorder it.
+// compiler cannot contract or reorder it.  The per-element quotients x / d
+// are not divided out one by one: a bracket of two products decides the code
+// and the exact division runs only where the bracket straddles a rounding
+// boundary (see `Bracket`).
 #include "bsq_common.cuh"
 
 namespace bsq {
@@ -44,11 +47,169 @@ __device__ __forceinline__ uint8_t f32_to_e4m3(float x) {
     return static_cast<uint8_t>(f32x2_to_e4m3x2(x, 0.0f) & 0xFF);
 }
 
-// Eight x / d quotients -> eight E2M1 nibbles in one 32-bit word, element 0
-// in the lowest nibble.
-__device__ __forceinline__ uint32_t nvfp4_codes_8(const uint4 &v, float d) {
+// Two E2M1 codes (one byte, element 2j in the low nibble) -> two FP32.
+__device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t byte) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.u8.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(h2)
+        : "r"(byte));
+    __half2 h = *reinterpret_cast<__half2 *>(&h2);
+    return __half22float2(h);
+}
+
+// Two E4M3 codes (low byte first) -> two FP32 (exact: every E4M3 value is an
+// FP16 value).
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t pair) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.u16.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h2)
+        : "r"(pair));
+    __half2 h = *reinterpret_cast<__half2 *>(&h2);
+    return __half22float2(h);
+}
+
+// ---------------------------------------------------------------------------
+// Codes of RN(x / d) without a division.
+//
+// Every code map used here (nearest E2M1 and nearest E4M3 with saturation,
+// nearest integer clamped to +-127; ties to even) is monotone in its FP32
+// argument and gives one code per value.  For d in [2^-60, 2^60] let r be
+// rcp.approx(d) (within 2^-23 of 1/d, relative), rl = RN(r (1 - 2^-16)) and
+// rh = RN(r (1 + 2^-16)).  Then RN(x rl) and RN(x rh) lie 2^-16 +- 2^-22 of
+// x/d away from it (relative), on opposite sides, while RN(x/d) is within
+// 2^-24 of it: RN(x/d) lies between the two products.  Quotients below
+// 2^-126, where relative bounds fail, round to a signed zero code in every
+// map, and so do the products then.  Hence:
+//   * both products give the same code: it is the code of RN(x/d);
+//   * they give two codes, necessarily adjacent (the bracket is far narrower
+//     than any gap between code boundaries).  The boundary m between them
+//     has few significant bits (3 for E2M1, 5 for E4M3; a half-integer for
+//     int8) and lies within 2^-15 of the products, so rounding a product to
+//     that many bits recovers it.  Then rho = x - m d is exact in one FMA
+//     (x and m d agree to 15 bits and their lowest bits lie no further
+//     apart than 24 bits), and (m of at most 8 bits) RN(x/d) = m exactly
+//     when |x|/d - |m| lies in [-h_in, h_out], h_out half an ulp of |m| and
+//     h_in the same except a quarter ulp where |m| is a power of two.  In
+//     that case the code map breaks the tie at m itself; otherwise the sign
+//     of rho picks the code above or below m.  All comparisons are exact:
+//     h d is a power-of-two multiple of d, normal in this range of d.
+// So the code of the correctly rounded quotient is found without dividing.
+//
+// Divisors with few significant bits need no bracket (see `snapped`).
+struct Bracket {
+    float r, lo, hi;
+    bool ok;
+};
+
+__device__ __forceinline__ Bracket bracket_of(float d) {
+    Bracket b;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(b.r) : "f"(d));
+    b.ok = d >= 0x1p-60f && d <= 0x1p60f;
+    b.lo = __fmul_rn(b.r, 1.0f - 0x1p-16f);
+    b.hi = __fmul_rn(b.r, 1.0f + 0x1p-16f);
+    return b;
+}
+
+// p rounded to B significant bits (round half up on the magnitude).
+template <int B>
+__device__ __forceinline__ float round_to_bits(float p) {
+    constexpr uint32_t half = 1u << (23 - B);
+    return __uint_as_float((__float_as_uint(p) + half) & ~(2u * half - 1u));
+}
+
+// Divisors with few significant bits.  Let x be BF16 (8 significant bits),
+// d have at most SB significant bits and every code boundary at most MB, with
+// SB + MB <= 9.  For x near 2^e and any MB-bit m with m d near x, x - m d is
+// a multiple of 2^(e-9), so x/d either equals m or lies at least 2^-10
+// (relative) from it.  p = RN(x r), r = rcp.approx(d), is within 2^-22 of
+// x/d.  So when p lies within 2^-12 of its rounding m to MB bits, x/d = m
+// exactly and RN(x/d) = m (the code map then breaks a tie at m itself);
+// otherwise no MB-bit number, and so no boundary, lies between p and
+// RN(x/d), and p has the code of RN(x/d).  is_short<SB> tests the bits of d.
+template <int MB>
+__device__ __forceinline__ float snapped(float p) {
+    const float m = round_to_bits<MB>(p);
+    const uint32_t ulps = __float_as_uint(p) - __float_as_uint(m) + 2048u;  // p, m share a sign
+    return ulps <= 4096u ? m : p;
+}
+
+template <int bits>
+__device__ __forceinline__ bool is_short(float d) {
+    return (__float_as_uint(d) & ((1u << (24 - bits)) - 1u)) == 0u;
+}
+
+// The half-integer nearest p (|p| < 2^21).
+__device__ __forceinline__ float nearest_half_integer(float p) {
+    const float a = __fadd_rn(__fadd_rn(__fadd_rn(fabsf(p), -0.5f), 12582912.0f), -12582912.0f);
+    return copysignf(__fadd_rn(a, 0.5f), p);
+}
+
+// A value whose code is the code of RN(x/d), for x/d next to the code
+// boundary m (see above).
+__device__ __forceinline__ float boundary_resolved(float x, float d, float m) {
+    const float rho = __fmaf_rn(-m, d, x);
+    if (rho == 0.0f) return m;  // x/d = m exactly
+    const uint32_t mb = __float_as_uint(m) & 0x7FFFFFFFu;
+    const float h_out = __fmul_rn(__uint_as_float(mb & 0x7F800000u), 0x1p-24f);
+    const float h_in = (mb & 0x7FFFFFu) ? h_out : __fmul_rn(h_out, 0.5f);
+    const float a = x < 0.0f ? -rho : rho;  // sign of |x|/d - |m|
+    if (a <= __fmul_rn(h_out, d) && a >= -__fmul_rn(h_in, d)) return m;
+    return __fmul_rn(m, a > 0.0f ? 1.0f + 0x1p-10f : 1.0f - 0x1p-10f);
+}
+
+// Codes (E2M1 or E4M3, by B) of a pair of quotients from their bracket ends:
+// p0, p1 the low-end products, lo/hi the code pairs of the two ends (FMT
+// bits per code).
+template <int B, int FMT>
+__device__ __forceinline__ void pair_boundaries(float x0, float x1, float d, float &p0, float &p1, uint32_t lo,
+                                                uint32_t hi) {
+    constexpr uint32_t mask = (1u << FMT) - 1u;
+    if ((lo ^ hi) & mask) p0 = boundary_resolved(x0, d, round_to_bits<B>(p0));
+    if ((lo ^ hi) >> FMT) p1 = boundary_resolved(x1, d, round_to_bits<B>(p1));
+}
+
+// E4M3 code of RN(x / d) for a BF16 x (the NVFP4 block scale).
+__device__ __forceinline__ uint8_t e4m3_of_quotient(float x, float d, const Bracket &br) {
+    if (!br.ok) return f32_to_e4m3(__fdiv_rn(x, d));
+    if (is_short<4>(d)) return f32_to_e4m3(snapped<5>(__fmul_rn(x, br.r)));
+    const float pl = __fmul_rn(x, br.lo), ph = __fmul_rn(x, br.hi);
+    const uint32_t b2 = f32x2_to_e4m3x2(pl, ph);
+    if ((b2 & 0xFFu) == (b2 >> 8)) return (uint8_t)(b2 & 0xFFu);
+    return f32_to_e4m3(boundary_resolved(x, d, round_to_bits<5>(pl)));
+}
+
+// Eight x / d quotients (packed BF16 x) -> eight E2M1 nibbles in one 32-bit
+// word, element 0 in the lowest nibble.
+__device__ __forceinline__ uint32_t nvfp4_codes_8(const uint4 &v, float d, const Bracket &br) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t out = 0;
+    if (br.ok && is_short<6>(d)) {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float p0 = __fmul_rn(lo_bf16(w[j]), br.r), p1 = __fmul_rn(hi_bf16(w[j]), br.r);
+            out |= f32x2_to_e2m1x2(snapped<3>(p0), snapped<3>(p1)) << (8 * j);
+        }
+        return out;
+    }
+    if (br.ok) {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float e0 = lo_bf16(w[j]), e1 = hi_bf16(w[j]);
+            float p0 = __fmul_rn(e0, br.lo), p1 = __fmul_rn(e1, br.lo);
+            uint32_t lo = f32x2_to_e2m1x2(p0, p1);
+            const uint32_t hi = f32x2_to_e2m1x2(__fmul_rn(e0, br.hi), __fmul_rn(e1, br.hi));
+            if (lo != hi) {
+                pair_boundaries<3, 4>(e0, e1, d, p0, p1, lo, hi);
+                lo = f32x2_to_e2m1x2(p0, p1);
+            }
+            out |= lo << (8 * j);
+        }
+        return out;
+    }
 #pragma unroll
     for (int j = 0; j < 4; j++) {
         float lo = __fdiv_rn(lo_bf16(w[j]), d);
@@ -58,22 +219,27 @@ __device__ __forceinline__ uint32_t nvfp4_codes_8(const uint4 &v, float d) {
     return out;
 }
 
-// Two threads per 16-element block, eight elements (16 bytes) each.
-__global__ void __launch_bounds__(256) k_quant_nvfp4(const uint16_t *__restrict__ in, uint32_t *__restrict__ packed,
+// One thread per 16-element block: two 16-byte loads, the block amax in
+// registers, eight code bytes and one scale byte stored.
+__global__ void __launch_bounds__(256) k_quant_nvfp4(const uint4 *__restrict__ in, uint2 *__restrict__ packed,
                                                      uint8_t *__restrict__ sf, float scale2, float t6,
-                                                     int64_t nhalf) {
+                                                     int64_t nblocks) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t h = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; h < nhalf; h += stride) {
-        const uint4 v = ld_nc_v4(in + h * 8);
-        uint32_t mx = amax_bits_8(v);
-        mx = max(mx, __shfl_xor_sync(__activemask(), mx, 1));
-        const float amax = __uint_as_float(mx << 16);
-        const uint8_t sc = f32_to_e4m3(__fdiv_rn(amax, t6));
+    const Bracket t6b = bracket_of(t6);
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+        const uint4 v0 = ld_nc_v4(in + 2 * b), v1 = ld_nc_v4(in + 2 * b + 1);
+        const uint32_t mx = max(amax_bits_8(v0), amax_bits_8(v1));
+        const uint8_t sc = e4m3_of_quotient(__uint_as_float(mx << 16), t6, t6b);
         const float sfv = e4m3_to_f32(sc);
-        uint32_t codes = 0;
-        if (sfv != 0.0f) codes = nvfp4_codes_8(v, __fmul_rn(sfv, scale2));
-        packed[h] = codes;
-        if ((h & 1) == 0) sf[h >> 1] = sc;
+        uint2 codes = make_uint2(0u, 0u);
+        if (sfv != 0.0f) {
+            const float d = __fmul_rn(sfv, scale2);
+            const Bracket br = bracket_of(d);
+            codes.x = nvfp4_codes_8(v0, d, br);
+            codes.y = nvfp4_codes_8(v1, d, br);
+        }
+        packed[b] = codes;
+        sf[b] = sc;
     }
 }
 
@@ -98,11 +264,25 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t *red) {
     return v;
 }
 
-// Eight E4M3 codes of x / s (RNE, satfinite) packed little-endian.
-__device__ __forceinline__ uint2 e4m3_codes_8(const float (&x)[8], float s) {
+// Eight E4M3 codes of x / s (RNE, satfinite) packed little-endian; `br` is
+// bracket_of(s).
+__device__ __forceinline__ uint2 e4m3_codes_8(const float (&x)[8], float s, const Bracket &br) {
     uint32_t w[4];
+    if (br.ok) {
 #pragma unroll
-    for (int j = 0; j < 4; j++) w[j] = f32x2_to_e4m3x2(__fdiv_rn(x[2 * j], s), __fdiv_rn(x[2 * j + 1], s));
+        for (int j = 0; j < 4; j++) {
+            float p0 = __fmul_rn(x[2 * j], br.lo), p1 = __fmul_rn(x[2 * j + 1], br.lo);
+            w[j] = f32x2_to_e4m3x2(p0, p1);
+            const uint32_t hi = f32x2_to_e4m3x2(__fmul_rn(x[2 * j], br.hi), __fmul_rn(x[2 * j + 1], br.hi));
+            if (w[j] != hi) {
+                pair_boundaries<5, 8>(x[2 * j], x[2 * j + 1], s, p0, p1, w[j], hi);
+                w[j] = f32x2_to_e4m3x2(p0, p1);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; j++) w[j] = f32x2_to_e4m3x2(__fdiv_rn(x[2 * j], s), __fdiv_rn(x[2 * j + 1], s));
+    }
     return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
@@ -111,48 +291,76 @@ __device__ __forceinline__ void unpack_bf16_8(const uint4 &v, float (&x)[8]) {
     x[4] = lo_bf16(v.z); x[5] = hi_bf16(v.z); x[6] = lo_bf16(v.w); x[7] = hi_bf16(v.w);
 }
 
-__device__ __forceinline__ uint2 row_codes_8(const uint4 &v, float s) {
+__device__ __forceinline__ uint2 row_codes_8(const uint4 &v, float s, const Bracket &br) {
     if (s == 0.0f) return make_uint2(0, 0);
     float f[8];
     unpack_bf16_8(v, f);
-    return e4m3_codes_8(f, s);
+    return e4m3_codes_8(f, s, br);
 }
 
-// One CTA per row: pass 1 finds the row amax (values kept in registers for
-// rows of up to NT*8*CH elements, re-read from cache beyond), pass 2 writes
-// the codes.
-constexpr int kRowThreads = 256;
-constexpr int kRowCh = 4;
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// Max over the CTA of a non-negative value held as float bits; one barrier
+// (the CTA handles a single row, so `red` is not reused).
+template <int NT>
+__device__ __forceinline__ uint32_t cta_max_once(uint32_t v, uint32_t *red) {
+    v = warp_max_u32(v);
+    if (NT == 32) return v;
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    v = red[0];
+#pragma unroll
+    for (int i = 1; i < NT / 32; i++) v = max(v, red[i]);
+    return v;
+}
+
+// Row-wise FP8: one CTA of kRowThreads per row.  Pass 1 finds the row amax
+// with the row's 16-byte chunks kept in registers (kRowKeep per thread, so
+// rows of up to kRowThreads * kRowKeep * 8 elements; longer rows are read
+// again in pass 2), pass 2 writes the codes.
+#ifndef BSQ_ROW_THREADS
+#define BSQ_ROW_THREADS 128
+#endif
+#ifndef BSQ_ROW_KEEP
+#define BSQ_ROW_KEEP 5
+#endif
+constexpr int kRowThreads = BSQ_ROW_THREADS;
+constexpr int kRowKeep = BSQ_ROW_KEEP;
 
 __global__ void __launch_bounds__(kRowThreads) k_quant_rowwise_fp8(const uint16_t *__restrict__ in,
                                                                    uint8_t *__restrict__ q,
                                                                    float *__restrict__ scale, int k) {
-    __shared__ uint32_t red[32];
+    __shared__ uint32_t red[kRowThreads / 32];
     const int64_t row = blockIdx.x;
+    const int t = threadIdx.x;
     const uint16_t *x = in + row * k;
     const int nch = k >> 3;
-    uint4 keep[kRowCh];
+    uint4 keep[kRowKeep];
     uint32_t mx = 0;
 #pragma unroll
-    for (int i = 0; i < kRowCh; i++) {
-        const int c = threadIdx.x + i * kRowThreads;
-        keep[i] = make_uint4(0, 0, 0, 0);
-        if (c < nch) keep[i] = ld_nc_v4(x + c * 8);
+    for (int i = 0; i < kRowKeep; i++) {
+        const int c = t + kRowThreads * i;
+        keep[i] = c < nch ? ld_nc_v4(x + c * 8) : make_uint4(0, 0, 0, 0);
         mx = max(mx, amax_bits_8(keep[i]));
     }
-    for (int c = threadIdx.x + kRowCh * kRowThreads; c < nch; c += kRowThreads) mx = max(mx, amax_bits_8(ld_nc_v4(x + c * 8)));
-    mx = block_max_u32<kRowThreads>(mx, red);
-    const float amax = __uint_as_float(mx << 16);
-    const float s = __fdiv_rn(amax, 448.0f);
-    if (threadIdx.x == 0) scale[row] = s;
+    for (int c = t + kRowThreads * kRowKeep; c < nch; c += kRowThreads)
+        mx = max(mx, amax_bits_8(ld_nc_v4(x + c * 8)));
+    mx = cta_max_once<kRowThreads>(mx, red);
+    const float s = __fdiv_rn(__uint_as_float(mx << 16), 448.0f);
+    if (t == 0) scale[row] = s;
+    const Bracket br = bracket_of(s);
     uint8_t *qr = q + row * k;
 #pragma unroll
-    for (int i = 0; i < kRowCh; i++) {
-        const int c = threadIdx.x + i * kRowThreads;
-        if (c < nch) *reinterpret_cast<uint2 *>(qr + c * 8) = row_codes_8(keep[i], s);
+    for (int i = 0; i < kRowKeep; i++) {
+        const int c = t + kRowThreads * i;
+        if (c < nch) *reinterpret_cast<uint2 *>(qr + c * 8) = row_codes_8(keep[i], s, br);
     }
-    for (int c = threadIdx.x + kRowCh * kRowThreads; c < nch; c += kRowThreads)
-        *reinterpret_cast<uint2 *>(qr + c * 8) = row_codes_8(ld_nc_v4(x + c * 8), s);
+    for (int c = t + kRowThreads * kRowKeep; c < nch; c += kRowThreads)
+        *reinterpret_cast<uint2 *>(qr + c * 8) = row_codes_8(ld_nc_v4(x + c * 8), s, br);
 }
 
 // One CTA per 128x128 block; 256 threads x 64 elements.
@@ -173,6 +381,7 @@ __global__ void __launch_bounds__(256) k_quant_blockfp8(const uint16_t *__restri
     mx = block_max_u32<256>(mx, red);
     const float s = __fdiv_rn(__uint_as_float(mx << 16), 448.0f);
     if (threadIdx.x == 0) scale[(int64_t)bi * gridDim.x + bj] = s;
+    const Bracket br = bracket_of(s);
     uint8_t *qo = q + ((int64_t)bi * 128 + r) * k + (int64_t)bj * 128 + c0;
 #pragma unroll
     for (int i = 0; i < 8; i++) {
@@ -180,137 +389,184 @@ __global__ void __launch_bounds__(256) k_quant_blockfp8(const uint16_t *__restri
         if (s != 0.0f) {
             float f[8];
             unpack_bf16_8(v[i], f);
-            out = e4m3_codes_8(f, s);
+            out = e4m3_codes_8(f, s, br);
         }
         *reinterpret_cast<uint2 *>(qo + i * 8) = out;
     }
 }
 
-// Block-scaled FP8 -> BF16 transient -> row-wise FP8, one CTA per row.  The
-// transient b = BF16(e4m3(w) * S) is recomputed in pass 2 instead of stored.
-__device__ __forceinline__ void dequant_16(const uint4 &w, float S, float (&b)[16]) {
+// Block-scaled FP8 -> BF16 transient -> row-wise FP8.  The transient
+// b = BF16(RN(e4m3(w) * S)) of a 16-code chunk is held packed (eight BF16x2
+// words) between the amax pass and the code pass; it is never stored.
+struct Bf16x16 {
+    uint4 a, b;  // elements 0-7, 8-15
+};
+
+__device__ __forceinline__ Bf16x16 dequant_16(const uint4 &w, float S) {
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[8];
 #pragma unroll
-    for (int j = 0; j < 16; j++) {
-        const uint8_t code = (ws[j >> 2] >> (8 * (j & 3))) & 0xFF;
-        const float p = __fmul_rn(e4m3_to_f32(code), S);
-        b[j] = __bfloat162float(__float2bfloat16_rn(p));
+    for (int j = 0; j < 8; j++) {
+        const float2 f = e4m3x2_to_f32x2((ws[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);  // exact
+        o[j] = pack_bf16x2(__fmul_rn(f.x, S), __fmul_rn(f.y, S));
     }
+    return {make_uint4(o[0], o[1], o[2], o[3]), make_uint4(o[4], o[5], o[6], o[7])};
 }
 
-__global__ void __launch_bounds__(kRowThreads) k_requant_blockfp8_to_rowwise(const uint8_t *__restrict__ w,
+__device__ __forceinline__ uint4 requant_codes_16(const Bf16x16 &t, float s, const Bracket &br) {
+    if (s == 0.0f) return make_uint4(0, 0, 0, 0);
+    float lo[8], hi[8];
+    unpack_bf16_8(t.a, lo);
+    unpack_bf16_8(t.b, hi);
+    const uint2 a = e4m3_codes_8(lo, s, br), b = e4m3_codes_8(hi, s, br);
+    return make_uint4(a.x, a.y, b.x, b.y);
+}
+
+// One CTA of kReqThreads per row, the row's transients kept in registers
+// (kReqKeep chunks per thread; longer rows are dequantised again).
+#ifndef BSQ_REQ_THREADS
+#define BSQ_REQ_THREADS 256
+#endif
+#ifndef BSQ_REQ_KEEP
+#define BSQ_REQ_KEEP 2
+#endif
+constexpr int kReqThreads = BSQ_REQ_THREADS;
+constexpr int kReqKeep = BSQ_REQ_KEEP;
+
+__global__ void __launch_bounds__(kReqThreads) k_requant_blockfp8_to_rowwise(const uint8_t *__restrict__ w,
                                                                              const float *__restrict__ bscale,
                                                                              uint8_t *__restrict__ q,
                                                                              float *__restrict__ scale, int k) {
-    __shared__ uint32_t red[32];
+    __shared__ uint32_t red[kReqThreads / 32];
     const int64_t row = blockIdx.x;
+    const int t = threadIdx.x;
     const int kb = k >> 7;
-    const float *srow = bscale + (row >> 7) * kb;
+    const float *srow = bscale + (row >> 7) * kb;  // one scale per 128 codes = 8 chunks
     const uint8_t *wr = w + row * k;
-    const int nch = k >> 4;  // 16 codes per chunk
+    const int nch = k >> 4;
+    Bf16x16 keep[kReqKeep];
     uint32_t mx = 0;
-    for (int c = threadIdx.x; c < nch; c += kRowThreads) {
-        float b[16];
-        dequant_16(ld_nc_v4(wr + c * 16), __ldg(srow + (c >> 3)), b);
 #pragma unroll
-        for (int j = 0; j < 16; j++) mx = max(mx, __float_as_uint(fabsf(b[j])));
+    for (int i = 0; i < kReqKeep; i++) {
+        const int c = t + kReqThreads * i;
+        keep[i] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        if (c < nch) keep[i] = dequant_16(ld_nc_v4(wr + c * 16), __ldg(srow + (c >> 3)));
+        mx = max(mx, max(amax_bits_8(keep[i].a), amax_bits_8(keep[i].b)));
     }
-    mx = block_max_u32<kRowThreads>(mx, red);
-    const float s = __fdiv_rn(__uint_as_float(mx), 448.0f);
-    if (threadIdx.x == 0) scale[row] = s;
+    for (int c = t + kReqThreads * kReqKeep; c < nch; c += kReqThreads) {
+        const Bf16x16 d = dequant_16(ld_nc_v4(wr + c * 16), __ldg(srow + (c >> 3)));
+        mx = max(mx, max(amax_bits_8(d.a), amax_bits_8(d.b)));
+    }
+    mx = cta_max_once<kReqThreads>(mx, red);
+    const float s = __fdiv_rn(__uint_as_float(mx << 16), 448.0f);
+    if (t == 0) scale[row] = s;
+    const Bracket br = bracket_of(s);
     uint8_t *qr = q + row * k;
-    for (int c = threadIdx.x; c < nch; c += kRowThreads) {
-        uint4 out = make_uint4(0, 0, 0, 0);
-        if (s != 0.0f) {
-            float b[16];
-            dequant_16(ld_nc_v4(wr + c * 16), __ldg(srow + (c >> 3)), b);
-            float lo[8], hi[8];
 #pragma unroll
-            for (int j = 0; j < 8; j++) { lo[j] = b[j]; hi[j] = b[8 + j]; }
-            const uint2 a = e4m3_codes_8(lo, s), bb = e4m3_codes_8(hi, s);
-            out = make_uint4(a.x, a.y, bb.x, bb.y);
-        }
-        *reinterpret_cast<uint4 *>(qr + c * 16) = out;
+    for (int i = 0; i < kReqKeep; i++) {
+        const int c = t + kReqThreads * i;
+        if (c < nch) *reinterpret_cast<uint4 *>(qr + c * 16) = requant_codes_16(keep[i], s, br);
     }
+    for (int c = t + kReqThreads * kReqKeep; c < nch; c += kReqThreads)
+        *reinterpret_cast<uint4 *>(qr + c * 16) =
+            requant_codes_16(dequant_16(ld_nc_v4(wr + c * 16), __ldg(srow + (c >> 3))), s, br);
 }
 
 // ---------------------------------------------------------------------------
 // int8 per-32 blocks, one thread per block.
 
-// Two E2M1 codes (one byte, element 2j in the low nibble) -> two FP32.
-__device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t byte) {
-    uint32_t h2;
-    asm("{\n\t.reg .b8 t;\n\t"
-        "cvt.u8.u32 t, %1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-        : "=r"(h2)
-        : "r"(byte));
-    __half2 h = *reinterpret_cast<__half2 *>(&h2);
-    return __half22float2(h);
+// Nearest integer (ties to even) of q clamped to [-127, 127], as the low
+// byte of the FP32 sum t + 1.5 * 2^23: in [2^23, 2^24) one unit is one ulp,
+// so the round-to-nearest addition rounds t itself.  Clamping before
+// rounding equals clamping after, the bounds being integers.
+__device__ __forceinline__ uint32_t int8_code_bits(float q) {
+    const float t = fminf(fmaxf(q, -127.0f), 127.0f);
+    return __float_as_uint(__fadd_rn(t, 12582912.0f));
 }
 
-__device__ __forceinline__ void int8_block_store(const float (&v)[32], int8_t *q, float *s_out) {
-    float amax = 0.0f;
+// Eight int8 codes of v / s packed little-endian (element 0 in the lowest
+// byte); `br` is bracket_of(s), s = RN(amax / 127) with |v| <= amax.  In the
+// bracketed range of s every product |v| r(1 +- 2^-16) stays below 127.5,
+// so the codes need no clamp: the low byte of RN(p + 1.5 * 2^23) is the
+// nearest integer of p (ties to even) in two's complement.
+__device__ __forceinline__ uint2 int8_codes_8(const float (&v)[8], float s, const Bracket &br) {
+    if (s == 0.0f) return make_uint2(0u, 0u);
+    uint32_t c[8];
+    if (br.ok) {
+        uint32_t h[8], diff = 0;
 #pragma unroll
-    for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
-    const float s = __fdiv_rn(amax, 127.0f);
-    *s_out = s;
-    uint32_t w[8];
-#pragma unroll
-    for (int j = 0; j < 8; j++) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; b++) {
-            int iv = 0;
-            if (s != 0.0f) {
-                const float r = fminf(fmaxf(rintf(__fdiv_rn(v[4 * j + b], s)), -127.0f), 127.0f);
-                iv = __float2int_rn(r);
-            }
-            word |= (static_cast<uint32_t>(iv) & 0xFFu) << (8 * b);
+        for (int i = 0; i < 8; i++) {
+            c[i] = __float_as_uint(__fadd_rn(__fmul_rn(v[i], br.lo), 12582912.0f));
+            h[i] = __float_as_uint(__fadd_rn(__fmul_rn(v[i], br.hi), 12582912.0f));
+            diff |= c[i] ^ h[i];
         }
-        w[j] = word;
+        if (diff != 0) {
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                if (c[i] != h[i])
+                    c[i] = int8_code_bits(
+                        boundary_resolved(v[i], s, nearest_half_integer(__fmul_rn(v[i], br.lo))));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; i++) c[i] = int8_code_bits(__fdiv_rn(v[i], s));
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(q);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    // low bytes of c[0..3] and c[4..7]
+    const uint32_t w0 = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
+    const uint32_t w1 = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
+    return make_uint2(w0, w1);
 }
 
-__global__ void __launch_bounds__(128) k_requant_w_nvfp4_int8(const uint8_t *__restrict__ packed,
+// Both int8 kernels give four threads to each 32-element block, eight
+// elements per thread; the block amax is a two-step shuffle inside the
+// quad, and one thread of the quad stores the block scale.  The grid stride
+// is a multiple of four, so a quad stays together to the last iteration.
+__device__ __forceinline__ float quad_max(float a) {
+    const unsigned mask = __activemask();
+    a = fmaxf(a, __shfl_xor_sync(mask, a, 1));
+    return fmaxf(a, __shfl_xor_sync(mask, a, 2));
+}
+
+__global__ void __launch_bounds__(256) k_requant_w_nvfp4_int8(const uint32_t *__restrict__ packed,
                                                               const uint8_t *__restrict__ sf, float scale2,
-                                                              int8_t *__restrict__ q, float *__restrict__ scale,
-                                                              int64_t nblocks) {
+                                                              uint2 *__restrict__ q, float *__restrict__ scale,
+                                                              int64_t ngroups) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
-        // block b covers elements [32b, 32b+32) of the flattened [n, k] tensor
-        const uint4 p = ld_nc_v4(packed + b * 16);
-        const float s0 = e4m3_to_f32(sf[b * 2]), s1 = e4m3_to_f32(sf[b * 2 + 1]);
-        const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
-        float v[32];
+    for (int64_t h = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; h < ngroups; h += stride) {
+        // group h: elements [8h, 8h+8) of the flattened [n, k] weight; its
+        // NVFP4 scale is that of the 16-element block h / 2
+        const uint32_t p = __ldg(packed + h);
+        const float sfv = e4m3_to_f32(__ldg(sf + (h >> 1)));
+        float v[8];
+        float amax = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 16; j++) {
-            const float2 e = e2m1x2_to_f32x2((pw[j >> 2] >> (8 * (j & 3))) & 0xFF);
-            const float sfv = j < 8 ? s0 : s1;
+        for (int j = 0; j < 4; j++) {
+            const float2 e = e2m1x2_to_f32x2((p >> (8 * j)) & 0xFFu);
             v[2 * j] = __fmul_rn(__fmul_rn(e.x, sfv), scale2);
             v[2 * j + 1] = __fmul_rn(__fmul_rn(e.y, sfv), scale2);
+            amax = fmaxf(amax, fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1])));
         }
-        int8_block_store(v, q + b * 32, scale + b);
+        amax = quad_max(amax);
+        const float s = __fdiv_rn(amax, 127.0f);
+        q[h] = int8_codes_8(v, s, bracket_of(s));
+        if ((h & 3) == 0) scale[h >> 2] = s;
     }
 }
 
-__global__ void __launch_bounds__(128) k_quant_act_int8_per32(const uint16_t *__restrict__ a,
-                                                              int8_t *__restrict__ q, float *__restrict__ scale,
-                                                              int64_t nblocks) {
+__global__ void __launch_bounds__(256) k_quant_act_int8_per32(const uint16_t *__restrict__ a, uint2 *__restrict__ q,
+                                                              float *__restrict__ scale, int64_t ngroups) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
-        float v[32];
-#pragma unroll
-        for (int c = 0; c < 4; c++) {
-            float f[8];
-            unpack_bf16_8(ld_nc_v4(a + b * 32 + c * 8), f);
-#pragma unroll
-            for (int i = 0; i < 8; i++) v[c * 8 + i] = f[i];
-        }
-        int8_block_store(v, q + b * 32, scale + b);
+    for (int64_t h = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; h < ngroups; h += stride) {
+        const uint4 x = ld_nc_v4(a + h * 8);
+        float v[8];
+        unpack_bf16_8(x, v);
+        uint32_t mx = amax_bits_8(x);
+        const unsigned mask = __activemask();
+        mx = max(mx, __shfl_xor_sync(mask, mx, 1));
+        mx = max(mx, __shfl_xor_sync(mask, mx, 2));
+        const float s = __fdiv_rn(__uint_as_float(mx << 16), 127.0f);
+        q[h] = int8_codes_8(v, s, bracket_of(s));
+        if ((h & 3) == 0) scale[h >> 2] = s;
     }
 }
 
@@ -338,10 +594,11 @@ int grid_for(int64_t work, int threads) {
 
 cudaError_t launch_quant_nvfp4(const uint16_t *in, uint8_t *packed, uint8_t *scale, float scale2, int m, int k,
                                cudaStream_t s) {
-    const int64_t nhalf = (int64_t)m * k / 8;
+    const int64_t nblocks = (int64_t)m * k / 16;
     const float t6 = 6.0f * scale2;
-    k_quant_nvfp4<<<grid_for(nhalf, 256), 256, 0, s>>>(in, reinterpret_cast<uint32_t *>(packed), scale, scale2, t6,
-                                                       nhalf);
+    k_quant_nvfp4<<<grid_for(nblocks, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(in),
+                                                         reinterpret_cast<uint2 *>(packed), scale, scale2, t6,
+                                                         nblocks);
     note_launch();
     return cudaGetLastError();
 }
@@ -361,23 +618,24 @@ cudaError_t launch_quant_blockfp8(const uint16_t *in, uint8_t *q, float *scale, 
 
 cudaError_t launch_requant_blockfp8_to_rowwise(const uint8_t *w, const float *bscale, int n, int k, uint8_t *q,
                                                float *scale, cudaStream_t s) {
-    k_requant_blockfp8_to_rowwise<<<n, kRowThreads, 0, s>>>(w, bscale, q, scale, k);
+    k_requant_blockfp8_to_rowwise<<<n, kReqThreads, 0, s>>>(w, bscale, q, scale, k);
     note_launch();
     return cudaGetLastError();
 }
 
 cudaError_t launch_requant_w_nvfp4_int8(const uint8_t *packed, const uint8_t *sf, float scale2, int8_t *q,
                                         float *scale, int n, int k, cudaStream_t s) {
-    const int64_t nb = (int64_t)n * k / 32;
-    k_requant_w_nvfp4_int8<<<grid_for(nb, 128), 128, 0, s>>>(packed, sf, scale2, q, scale, nb);
+    const int64_t ng = (int64_t)n * k / 8;
+    k_requant_w_nvfp4_int8<<<grid_for(ng, 256), 256, 0, s>>>(reinterpret_cast<const uint32_t *>(packed), sf, scale2,
+                                                             reinterpret_cast<uint2 *>(q), scale, ng);
     note_launch();
     return cudaGetLastError();
 }
 
 cudaError_t launch_quant_act_int8_per32(const uint16_t *a, int8_t *q, float *scale, int m, int k,
                                         cudaStream_t s) {
-    const int64_t nb = (int64_t)m * k / 32;
-    k_quant_act_int8_per32<<<grid_for(nb, 128), 128, 0, s>>>(a, q, scale, nb);
+    const int64_t ng = (int64_t)m * k / 8;
+    k_quant_act_int8_per32<<<grid_for(ng, 256), 256, 0, s>>>(a, reinterpret_cast<uint2 *>(q), scale, ng);
     note_launch();
     return cudaGetLastError();
 }

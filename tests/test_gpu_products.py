@@ -54,7 +54,8 @@ def run_w4a4(ap, asf, wp, wsf, sa2, sb2):
     return host(out, np.uint16)
 
 
-@pytest.mark.parametrize("mnk", [(16, 256, 512), (200, 300, 512), (129, 520, 768), (1, 8, 256)])
+@pytest.mark.parametrize("mnk", [(16, 256, 512), (200, 300, 512), (129, 520, 768), (1, 8, 256), (300, 1000, 1024),
+                                 (257, 510, 1536)])
 def test_w4a4_small_and_ragged(mnk):
     m, n, k = mnk
     args = nvfp4_from_oracle(m, n, k, seed=1)

@@ -173,3 +173,127 @@ def test_amax_exact_and_empty():
     bsq.bsq_amax_bf16(None, 0, amax)
     torch.cuda.synchronize()
     assert float(amax.item()) == 0.0
+
+
+# ---------------------------------------------------------------------------
+# Rounding boundaries.  The kernels decide most codes from two products that
+# bracket the quotient and divide exactly only where the bracket straddles a
+# boundary between two codes; these rows put quotients exactly on the
+# boundaries (ties) and one BF16 step either side of them.
+
+def _e4m3_values():
+    sub = [m * 2.0 ** -9 for m in range(0, 8)]
+    nrm = [(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8) if not (e == 15 and m == 7)]
+    return np.array(sub + nrm, np.float64)
+
+
+def _bf16_exact(v):
+    b = synth.to_bf16_bits(np.asarray(v, np.float32))
+    back = (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(back, np.asarray(v, np.float64)), "boundary value not exact in BF16"
+    return b
+
+
+def _neighbours(v):
+    """v and the BF16 values one step below and above it (v > 0)."""
+    b = synth.to_bf16_bits(np.asarray(v, np.float32)).astype(np.int32)
+    out = np.stack([b - 1, b, b + 1], -1).reshape(-1).astype(np.uint16)
+    return (out.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def e4m3_boundary_rows(scales, k=256):
+    """One row per scale s: amax 448 s, then s times every E4M3 midpoint
+    and its BF16 neighbours, with alternating signs."""
+    vals = _e4m3_values()
+    mids = (vals[:-1] + vals[1:]) / 2
+    rows = []
+    for s in scales:
+        body = _neighbours(mids * s)
+        body = body * np.where(np.arange(body.size) % 2 == 0, 1.0, -1.0)
+        row = np.concatenate([[448.0 * s], body])
+        row = np.resize(row, k)
+        row[0] = 448.0 * s
+        _bf16_exact(row[:1])
+        rows.append(row)
+    return synth.to_bf16_bits(np.array(rows, np.float32))
+
+
+def test_quant_rowwise_fp8_rounding_boundaries():
+    x = e4m3_boundary_rows([1.0, 3.0, 0.75, 2.0 ** -6], k=1024)
+    m, k = x.shape
+    q, s = empty(x.shape, torch.uint8), empty((m,), torch.float32)
+    bsq.quant_rowwise_fp8(to_dev(x), q, s, m, k)
+    torch.cuda.synchronize()
+    oq, os_ = oracle.quant_rowwise_fp8(x)
+    assert np.array_equal(host(s), os_)
+    assert np.array_equal(host(q), oq), f"codes differ at {np.argwhere(host(q) != oq)[:4]}"
+
+
+def test_quant_blockfp8_rounding_boundaries():
+    rows = e4m3_boundary_rows([1.0, 3.0], k=256)
+    x = np.repeat(rows, 128, axis=0)  # 256 x 256: 2 x 2 blocks, amax 448 s in each
+    x = np.ascontiguousarray(x)
+    q, S = empty(x.shape, torch.uint8), empty((2, 2), torch.float32)
+    bsq.quant_blockfp8(to_dev(x), q, S, 256, 256)
+    torch.cuda.synchronize()
+    oq, oS = oracle.quant_blockfp8(x)
+    assert np.array_equal(host(S), oS)
+    assert np.array_equal(host(q), oq)
+
+
+def test_quant_act_int8_rounding_boundaries():
+    blocks = []
+    for s in (1.0, 2.0, 0.5):
+        halves = (np.arange(0, 127) + 0.5) * s
+        body = _neighbours(halves) * np.where(np.arange(3 * 127) % 2 == 0, 1.0, -1.0)
+        for c in range(0, body.size, 31):
+            blk = np.zeros(32)
+            blk[0] = 127.0 * s
+            seg = body[c:c + 31]
+            blk[1:1 + seg.size] = seg
+            blocks.append(blk)
+    while len(blocks) % 8:
+        blocks.append(blocks[0])
+    x = synth.to_bf16_bits(np.array(blocks, np.float32).reshape(-1, 256))
+    m, k = x.shape
+    q, s = empty(x.shape, torch.int8), empty((m, k // 32), torch.float32)
+    bsq.quant_act_int8_per32(to_dev(x), q, s, m, k)
+    torch.cuda.synchronize()
+    oq, os_ = oracle.quant_act_int8_per32(x)
+    assert np.array_equal(host(s), os_)
+    assert np.array_equal(host(q), oq), f"codes differ at {np.argwhere(host(q) != oq)[:4]}"
+
+
+def test_quant_nvfp4_scale_rounding_boundaries():
+    """Block amaxes at 6 x (every E4M3 midpoint up to 448), so that the scale
+    quotient amax / (6 scale2) is a tie, with E2M1 midpoints inside."""
+    vals = _e4m3_values()
+    mids = ((vals[:-1] + vals[1:]) / 2)[8:]  # normal range
+    blocks = []
+    for mu in mids:
+        amax = 6.0 * mu
+        blk = np.array([amax, -0.25, 0.75, -1.25, 1.75, -2.5, 3.5, -5.0, 0.5, 1, 2, 3, 4, -6, 0.3, 0.1]) * mu
+        blk[0] = amax
+        blocks.append(blk)
+    n = len(blocks) // 4 * 4
+    x = synth.to_bf16_bits(np.array(blocks[:n], np.float32).reshape(-1, 64))
+    gp, gs = gpu_nvfp4(x, 1.0)
+    op, os_ = oracle.quant_nvfp4(x, 1.0)
+    assert np.array_equal(gs, os_), f"scales differ at {np.argwhere(gs != os_)[:4]}"
+    assert np.array_equal(gp, op), f"codes differ at {np.argwhere(gp != op)[:4]}"
+
+
+@pytest.mark.parametrize("scale2", [1.0, 0.75, 0.625, 2.0 ** -3, float(np.float32(1 / 3)), 1e-3])
+def test_quant_nvfp4_divisor_classes(scale2):
+    """The block divisor d = e4m3(sf) * scale2 has few significant bits for
+    scale2 = 1, 0.75, 2^-3 (exact ties are then common and the kernel snaps
+    to the boundary) and many for 0.625 (7 bits with some scales), 1/3 and
+    1e-3 (the bracketed path).  Tie-heavy rows scaled by scale2 and
+    Student-t rows, bit-exact against the oracle."""
+    ties = (special_rows().astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    body = synth.student_t_bf16((64, 1024), 4.0, 4, 3, outlier_frac=0.01)
+    x = np.concatenate([synth.to_bf16_bits(np.resize(ties * scale2, (3, 1024)).astype(np.float32)), body])
+    gp, gs = gpu_nvfp4(x, scale2)
+    op, os_ = oracle.quant_nvfp4(x, scale2)
+    assert np.array_equal(gs, os_), f"scales differ at {np.argwhere(gs != os_)[:4]}"
+    assert np.array_equal(gp, op), f"codes differ at {np.argwhere(gp != op)[:4]}"
