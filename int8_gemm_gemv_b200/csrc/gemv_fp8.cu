@@ -4,8 +4,9 @@
 //   out[m, n] = row_scale[n] * sum_k bf16(in[m, k]) * e4m3(W[n, k])
 //
 // The weight stream (N*K bytes, read once) is the whole cost.  Design:
-//   * persistent: one CTA per SM, each owning a contiguous range of 16-row
-//     weight tiles (balanced to within one tile);
+//   * persistent: one CTA per SM, each owning a contiguous range of 8-row
+//     weight units (balanced to within 8 rows), streamed as 16-row tiles
+//     with a final 8-row tile where the count is odd;
 //   * warp 16 streams the CTA's weight rows with TMA into a 192 KB ring of
 //     stages (two 16-row tiles x 1024 K bytes each, 128-byte swizzle), so
 //     up to 192 KB of loads are in flight per SM: for a 5120 x 5120 weight
@@ -110,8 +111,9 @@ __device__ __forceinline__ uint32_t stage_offset(int u, int w, int r, int t) {
 
 template <int MT>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_fp8_gemv(const __grid_constant__ CUtensorMap tmW, const uint8_t *__restrict__ wptr, const uint16_t *__restrict__ X,
-               const float *__restrict__ row_scale, uint16_t *__restrict__ out, int M, int N, int K, int tm3d) {
+    k_fp8_gemv(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW8,
+               const uint8_t *__restrict__ wptr, const uint16_t *__restrict__ X, const float *__restrict__ row_scale,
+               uint16_t *__restrict__ out, int M, int N, int K, int tm3d) {
     extern __shared__ uint8_t smem_raw[];
     // the next kernel of the stream may start its own prologue now
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -120,9 +122,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     Smem *S = reinterpret_cast<Smem *>(red + kConsumers * 2 * MT * 4 * 32);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles = (N + 15) >> 4;
-    const int t_begin = (int)((int64_t)tiles * blockIdx.x / gridDim.x);
-    const int t_end = (int)((int64_t)tiles * (blockIdx.x + 1) / gridDim.x);
+    // this CTA's rows [row_begin, row_end): a range of 8-row units, taken as
+    // 16-row tiles, the last one 8 rows (its other 8 rows are neither loaded
+    // nor stored) when the unit count is odd
+    const int units = (N + 7) >> 3;
+    const int u_begin = (int)((int64_t)units * blockIdx.x / gridDim.x);
+    const int u_end = (int)((int64_t)units * (blockIdx.x + 1) / gridDim.x);
+    const int row_begin = 8 * u_begin, row_end = min(8 * u_end, N);
+    const int t_end = (u_end - u_begin + 1) >> 1;  // tiles, counted from 0
+    const bool half_last = ((u_end - u_begin) & 1) != 0;
     const int nst = (K + KS - 1) / KS;  // stages per tile pair
 
     if (threadIdx.x == 0) {
@@ -139,10 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         const uint8_t *wbase = reinterpret_cast<const uint8_t *>(wptr);
         uint64_t done = 0;
-        for (int t = t_begin; t < t_end && done < kPrefetchBytes; t++) {
-            const int rows = min(16, N - 16 * t);
+        for (int r = row_begin; r < row_end && done < kPrefetchBytes; r += 16) {
+            const int rows = min(16, row_end - r);
             const uint64_t bytes = (uint64_t)rows * K;
-            prefetch_l2_bulk(wbase + (uint64_t)t * 16 * K, (uint32_t)bytes);
+            prefetch_l2_bulk(wbase + (uint64_t)r * K, (uint32_t)bytes);
             done += bytes;
         }
     }
@@ -158,8 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tmW);
             uint32_t it = 0;
             bool ok = true;
-            for (int t0 = t_begin; t0 < t_end && ok; t0 += 2) {
+            for (int t0 = 0; t0 < t_end && ok; t0 += 2) {
                 const int nt = min(2, t_end - t0);
+                const bool half = half_last && t0 + nt == t_end;  // the pair's last tile has 8 rows
                 for (int q = 0; q < nst; q++, it++) {
                     const int s = it % STAGES;
                     if (!mbar_wait(&S->empty[s], ((it / STAGES) & 1) ^ 1, &g_timeouts) || S->abort) {
@@ -167,15 +176,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     uint8_t *st = base + (size_t)s * STAGE_BYTES;
-                    mbar_arrive_expect_tx(&S->full[s], nt * TILE_BYTES);
+                    mbar_arrive_expect_tx(&S->full[s], nt * TILE_BYTES - (half ? TILE_BYTES / 2 : 0));
                     for (int u = 0; u < nt; u++) {
-                        if (tm3d) {  // one copy: 16 rows x 8 chunks of 128 B
-                            tma_load_3d(st + u * TILE_BYTES, &tmW, &S->full[s], 0, (t0 + u) * 16, q * (KS / BOX));
+                        const int row0 = row_begin + 16 * (t0 + u);
+                        if (half && u == nt - 1) {  // 8 rows: eight 1 KB copies into the tile's first halves
+#pragma unroll
+                            for (int j = 0; j < KS / BOX; j++)
+                                tma_load_2d(st + u * TILE_BYTES + j * 16 * BOX, &tmW8, &S->full[s], q * KS + j * BOX,
+                                            row0);
+                        } else if (tm3d) {  // one copy: 16 rows x 8 chunks of 128 B
+                            tma_load_3d(st + u * TILE_BYTES, &tmW, &S->full[s], 0, row0, q * (KS / BOX));
                         } else {
 #pragma unroll
                             for (int j = 0; j < KS / BOX; j++)
                                 tma_load_2d(st + u * TILE_BYTES + j * 16 * BOX, &tmW, &S->full[s], q * KS + j * BOX,
-                                            (t0 + u) * 16);
+                                            row0);
                         }
                     }
                 }
@@ -201,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     uint32_t it = 0;
     bool ok = true;
-    for (int t0 = t_begin; t0 < t_end; t0 += 2) {
+    for (int t0 = 0; t0 < t_end; t0 += 2) {
         const int nt = min(2, t_end - t0);
         float acc[2][MT][4];
 #pragma unroll
@@ -276,9 +291,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int r = 0; r < 4; r++) v[r] += red[(((w * 2 + u) * MT + i) * 4 + r) * 32 + lane];
 #pragma unroll
             for (int r = 0; r < 4; r++) {
-                const int n = (t0 + u) * 16 + g + 8 * (r >> 1);
+                const int n = row_begin + (t0 + u) * 16 + g + 8 * (r >> 1);
                 const int m = 8 * i + 2 * t + (r & 1);
-                if (n < N && m < M)
+                if (n < row_end && m < M)
                     out[(int64_t)m * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v[r] * __ldg(row_scale + n)));
             }
         }
@@ -297,8 +312,9 @@ uint32_t take_timeouts_gemv() {
 }
 
 template <int MT>
-static cudaError_t launch_mt(const CUtensorMap &tm, int tm3d, const uint8_t *w, const uint16_t *in,
-                             const float *row_scale, uint16_t *out, int m, int n, int k, cudaStream_t s) {
+static cudaError_t launch_mt(const CUtensorMap &tm, const CUtensorMap &tm8, int tm3d, const uint8_t *w,
+                             const uint16_t *in, const float *row_scale, uint16_t *out, int m, int n, int k,
+                             cudaStream_t s) {
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -308,8 +324,8 @@ static cudaError_t launch_mt(const CUtensorMap &tm, int tm3d, const uint8_t *w, 
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    const int tiles = (n + 15) / 16;
-    const int grid = tiles < sm_count() ? tiles : sm_count();
+    const int units = (n + 7) / 8;
+    const int grid = units < sm_count() ? units : sm_count();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -320,20 +336,22 @@ static cudaError_t launch_mt(const CUtensorMap &tm, int tm3d, const uint8_t *w, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_fp8_gemv<MT>, tm, w, in, row_scale, out, m, n, k, tm3d);
+    return cudaLaunchKernelEx(&cfg, k_fp8_gemv<MT>, tm, tm8, w, in, row_scale, out, m, n, k, tm3d);
 }
 
 cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *row_scale, uint16_t *out,
                                      int m, int n, int k, cudaStream_t s) {
-    alignas(64) CUtensorMap tm;
+    alignas(64) CUtensorMap tm, tm8;
     // K a multiple of 128: one 16 KB copy per tile and stage; otherwise eight
-    // 2 KB copies (the last chunk of a row may be partial)
+    // 2 KB copies (the last chunk of a row may be partial).  8-row tiles:
+    // eight 1 KB copies.
     const int tm3d = (k % BOX) == 0;
-    const bool ok = tm3d ? make_tmap_rows_chunks(&tm, w, k, n, 16, KS / BOX)
-                         : make_tmap_2d(&tm, w, 1, k, n, k, BOX, 16, true, false);
+    const bool ok = (tm3d ? make_tmap_rows_chunks(&tm, w, k, n, 16, KS / BOX)
+                          : make_tmap_2d(&tm, w, 1, k, n, k, BOX, 16, true, false)) &&
+                    make_tmap_2d(&tm8, w, 1, k, n, k, BOX, 8, true, false);
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = m <= 8 ? launch_mt<1>(tm, tm3d, w, in, row_scale, out, m, n, k, s)
-                           : launch_mt<2>(tm, tm3d, w, in, row_scale, out, m, n, k, s);
+    cudaError_t e = m <= 8 ? launch_mt<1>(tm, tm8, tm3d, w, in, row_scale, out, m, n, k, s)
+                           : launch_mt<2>(tm, tm8, tm3d, w, in, row_scale, out, m, n, k, s);
     note_launch();
     return e;
 }
