@@ -171,6 +171,33 @@ def time_launches(torch, stream, fn, iters, warm=3):
     return s.elapsed_time(e) * 1e-3 / iters
 
 
+def time_graph(torch, fn, iters, reps=5):
+    """Average device time of fn(stream) over iters launches captured into
+    one CUDA graph and replayed reps times (events on the replay stream):
+    back-to-back kernel time without per-launch host overhead, for kernels
+    short enough for that overhead to matter."""
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        for _ in range(3):
+            fn(st)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        for _ in range(iters):
+            fn(st)
+    with torch.cuda.stream(st):
+        g.replay()
+        s, e = _events(torch, 2)
+        st.synchronize()
+        s.record(st)
+        for _ in range(reps):
+            g.replay()
+        e.record(st)
+    e.synchronize()
+    del g
+    return s.elapsed_time(e) * 1e-3 / (reps * iters)
+
+
 def kernel_hash(name):
     with open(os.path.join(ROOT, "int8_gemm_gemv_b200", "csrc", name), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
@@ -353,24 +380,36 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
             out = torch.empty((m, n), dtype=torch.int16, device=dev)
             it = [0]
 
-            def f():
+            def f(st):
                 wq, ws = ws_list[it[0] % len(ws_list)]
                 it[0] += 1
-                bsq.fp8_gemv_rowscale(x, wq, ws, out, m, n, k, stream)
-            t = time_launches(torch, stream, f, 200)
+                bsq.fp8_gemv_rowscale(x, wq, ws, out, m, n, k, st)
+            t = time_graph(torch, f, 4 * len(ws_list))
             hbm_row(f"a4_fp8_gemv_m{m}_n{n}_k{k}", t, n * k + 4 * n + 2 * m * k + 2 * m * n,
                     {"l2": f"{len(ws_list)} rotating weight copies"})
         del ws_list
         torch.cuda.empty_cache()
 
-    # a1: NVFP4 quantiser, 4096x5120 and 16384x5120
+    def rotating(fn_of, inputs, reps_per_input=4):
+        """fn(stream) cycling through the input copies."""
+        it = [0]
+
+        def f(st):
+            fn_of(inputs[it[0] % len(inputs)], st)
+            it[0] += 1
+        return f, reps_per_input * len(inputs)
+
+    # a1: NVFP4 quantiser, 4096x5120 and 16384x5120 (inputs rotated past L2)
     for m in (4096, 16384):
         k = 5120
-        a = bf16_rand((m, k), 1.0)
+        a_list = rotate(lambda: bf16_rand((m, k), 1.0), m * k * 2)
         ap = torch.empty((m, k // 2), dtype=torch.uint8, device=dev)
         asf = torch.empty((m, k // 16), dtype=torch.uint8, device=dev)
-        t = time_launches(torch, stream, lambda: bsq.quantize_bf16_to_nvfp4(a, ap, asf, 1.0, m, k, stream), 50)
-        hbm_row(f"a1_quantize_bf16_to_nvfp4_{m}x{k}", t, m * k * 2 + m * k // 2 + m * k // 16)
+        f, n_it = rotating(lambda a, st: bsq.quantize_bf16_to_nvfp4(a, ap, asf, 1.0, m, k, st), a_list)
+        t = time_graph(torch, f, n_it)
+        hbm_row(f"a1_quantize_bf16_to_nvfp4_{m}x{k}", t, m * k * 2 + m * k // 2 + m * k // 16,
+                {"l2": f"{len(a_list)} rotating input copies"})
+        del a_list
 
     # a2: W4A4 GEMM at M = 512 and 16384 (4096 is the headline step)
     n, k = 17408, 5120
@@ -389,23 +428,36 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
 
     # a3: row-wise FP8 quantiser (per-token activations of the FP8 projection)
     m, k = 8192, 5120
-    a = bf16_rand((m, k), 1.0)
+    a_list = rotate(lambda: bf16_rand((m, k), 1.0), m * k * 2)
     q = torch.empty((m, k), dtype=torch.uint8, device=dev)
     s = torch.empty((m,), dtype=torch.float32, device=dev)
-    t = time_launches(torch, stream, lambda: bsq.quant_rowwise_fp8(a, q, s, m, k, stream), 50)
-    hbm_row(f"a3_quant_rowwise_fp8_{m}x{k}", t, m * k * 3 + 4 * m)
+    f, n_it = rotating(lambda a, st: bsq.quant_rowwise_fp8(a, q, s, m, k, st), a_list)
+    t = time_graph(torch, f, n_it)
+    hbm_row(f"a3_quant_rowwise_fp8_{m}x{k}", t, m * k * 3 + 4 * m, {"l2": f"{len(a_list)} rotating input copies"})
+    a = a_list[0]
+    bsq.quant_rowwise_fp8(a, q, s, m, k, stream)
+    del a_list
 
     # a8: block FP8 -> row-wise FP8 requant (one-time weight conversion)
     n, k = 10240, 5120
     wsrc = bf16_rand((n, k), 0.02)
-    wb = torch.empty((n, k), dtype=torch.uint8, device=dev)
-    S = torch.empty((n // 128, k // 128), dtype=torch.float32, device=dev)
-    bsq.quant_blockfp8(wsrc, wb, S, n, k, stream)
+
+    def mk_block():
+        wb = torch.empty((n, k), dtype=torch.uint8, device=dev)
+        S = torch.empty((n // 128, k // 128), dtype=torch.float32, device=dev)
+        bsq.quant_blockfp8(wsrc, wb, S, n, k, stream)
+        return wb, S
+    blk_list = rotate(mk_block, n * k)
     wr = torch.empty((n, k), dtype=torch.uint8, device=dev)
     sr = torch.empty((n,), dtype=torch.float32, device=dev)
-    t = time_launches(torch, stream, lambda: bsq.requant_blockfp8_to_rowwise(
-        bsq.BSQ_FP8_BLOCK_SCALED, wb, S, n, k, wr, sr, stream), 20)
-    hbm_row(f"a8_requant_blockfp8_to_rowwise_{n}x{k}", t, 2 * n * k + 4 * n + 4 * (n // 128) * (k // 128))
+    f, n_it = rotating(lambda b, st: bsq.requant_blockfp8_to_rowwise(
+        bsq.BSQ_FP8_BLOCK_SCALED, b[0], b[1], n, k, wr, sr, st), blk_list)
+    t = time_graph(torch, f, n_it)
+    hbm_row(f"a8_requant_blockfp8_to_rowwise_{n}x{k}", t, 2 * n * k + 4 * n + 4 * (n // 128) * (k // 128),
+            {"l2": f"{len(blk_list)} rotating input copies"})
+    wb, S = blk_list[0]
+    bsq.requant_blockfp8_to_rowwise(bsq.BSQ_FP8_BLOCK_SCALED, wb, S, n, k, wr, sr, stream)
+    del blk_list
 
     # a9: row-scaled FP8 GEMM 8192 x 10240 x 5120
     m = 8192
@@ -419,18 +471,31 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
     # a5 / a6 / a7: the W4A8 int8 path
     n, k, m = 5120, 17408, 2048
     wsrc = bf16_rand((n, k), 0.02)
-    wp = torch.empty((n, k // 2), dtype=torch.uint8, device=dev)
-    wsf = torch.empty((n, k // 16), dtype=torch.uint8, device=dev)
-    bsq.quantize_bf16_to_nvfp4(wsrc, wp, wsf, 1e-5, n, k, stream)
+
+    def mk_nvfp4():
+        wp = torch.empty((n, k // 2), dtype=torch.uint8, device=dev)
+        wsf = torch.empty((n, k // 16), dtype=torch.uint8, device=dev)
+        bsq.quantize_bf16_to_nvfp4(wsrc, wp, wsf, 1e-5, n, k, stream)
+        return wp, wsf
+    w_list = rotate(mk_nvfp4, n * k // 2)
+    del wsrc
     wi = torch.empty((n, k), dtype=torch.int8, device=dev)
     wis = torch.empty((n, k // 32), dtype=torch.float32, device=dev)
-    t = time_launches(torch, stream, lambda: bsq.requant_w_nvfp4_int8(wp, wsf, 1e-5, wi, wis, n, k, stream), 20)
-    hbm_row(f"a5_requant_w_nvfp4_int8_{n}x{k}", t, n * k // 2 + n * k // 16 + n * k + n * k // 8)
-    a = bf16_rand((m, k), 1.0)
+    f, n_it = rotating(lambda wq, st: bsq.requant_w_nvfp4_int8(wq[0], wq[1], 1e-5, wi, wis, n, k, st), w_list, 2)
+    t = time_graph(torch, f, n_it, reps=3)
+    hbm_row(f"a5_requant_w_nvfp4_int8_{n}x{k}", t, n * k // 2 + n * k // 16 + n * k + n * k // 8,
+            {"l2": f"{len(w_list)} rotating input copies"})
+    wp, wsf = w_list[0]
+    bsq.requant_w_nvfp4_int8(wp, wsf, 1e-5, wi, wis, n, k, stream)
+    del w_list
+    a_list = rotate(lambda: bf16_rand((m, k), 1.0), m * k * 2)
     ai = torch.empty((m, k), dtype=torch.int8, device=dev)
     ais = torch.empty((m, k // 32), dtype=torch.float32, device=dev)
-    t = time_launches(torch, stream, lambda: bsq.quant_act_int8_per32(a, ai, ais, m, k, stream), 50)
-    hbm_row(f"a6_quant_act_int8_per32_{m}x{k}", t, m * k * 3 + m * k // 8)
+    f, n_it = rotating(lambda a, st: bsq.quant_act_int8_per32(a, ai, ais, m, k, st), a_list)
+    t = time_graph(torch, f, n_it)
+    hbm_row(f"a6_quant_act_int8_per32_{m}x{k}", t, m * k * 3 + m * k // 8, {"l2": f"{len(a_list)} rotating input copies"})
+    bsq.quant_act_int8_per32(a_list[0], ai, ais, m, k, stream)
+    del a_list
     out = torch.empty((m, n), dtype=torch.int16, device=dev)
     t = time_launches(torch, stream, lambda: bsq.int8_blockscaled_gemm(ai, wi, ais, wis, out, m, n, k, stream), 5)
     tops = 2.0 * m * n * k / t / 1e12
