@@ -259,26 +259,33 @@ def run_bsq(args, w, peaks, peak_src):
 
     for i in range(args.warmup):
         step(i)
-    ev = _events(torch, 3 * args.steps)
     t0, t1 = _events(torch, 2)
     barrier(dev)
     launches0 = bsq.debug_launch_count()
+    # the timed region: back-to-back steps with no event between the two
+    # kernels, so the GEMM's prologue overlaps the quantiser's tail
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         t0.record(stream)
         for i in range(args.steps):
-            j = i % nsets
-            wp, wsf, sb2 = w_codes[j]
-            ev[3 * i].record(stream)
-            bsq.quantize_bf16_to_nvfp4(a_dev[j], ap[j], asf[j], 1.0, m, k, stream)
-            ev[3 * i + 1].record(stream)
-            bsq.w4a4_gemm(ap[j], asf[j], wp, wsf, out, 1.0, sb2, m, n, k, stream)
-            ev[3 * i + 2].record(stream)
+            step(i)
         t1.record(stream)
         t1.synchronize()
     launches = bsq.debug_launch_count() - launches0
     barrier(dev)
     elapsed = t0.elapsed_time(t1) * 1e-3
     t_max = max_over_ranks(elapsed, dev)
+    # per-kernel durations: the same steps again, each kernel between its
+    # own events (this serialises the two kernels of a step)
+    ev = _events(torch, 3 * args.steps)
+    for i in range(args.steps):
+        j = i % nsets
+        wp, wsf, sb2 = w_codes[j]
+        ev[3 * i].record(stream)
+        bsq.quantize_bf16_to_nvfp4(a_dev[j], ap[j], asf[j], 1.0, m, k, stream)
+        ev[3 * i + 1].record(stream)
+        bsq.w4a4_gemm(ap[j], asf[j], wp, wsf, out, 1.0, sb2, m, n, k, stream)
+        ev[3 * i + 2].record(stream)
+    ev[-1].synchronize()
     quant_t = statistics.mean(ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(args.steps)) * 1e-3
     gemm_t = statistics.mean(ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(args.steps)) * 1e-3
     flops = 2.0 * m * n * k
@@ -425,6 +432,22 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
                                       "frac_fp4": round(tf / (bf16 * RATIO_FP4), 4), "bound": "tensor"}
         del ap, asf, out
     del wp, wsf
+    # a2, few activation rows (swapped-operand kernel): the weight stream
+    # (N*K/2 + N*K/16 bytes) is the cost; weight copies rotated past L2
+    def mk_w4():
+        return (torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=dev, generator=g),
+                torch.randint(0x30, 0x40, (n, k // 16), dtype=torch.uint8, device=dev, generator=g))
+    w4_list = rotate(mk_w4, n * k // 2 + n * k // 16)
+    for m in (1, 16, 128):
+        ap = torch.randint(0, 256, (m, k // 2), dtype=torch.uint8, device=dev, generator=g)
+        asf = torch.randint(0x30, 0x40, (m, k // 16), dtype=torch.uint8, device=dev, generator=g)
+        out = torch.empty((m, n), dtype=torch.int16, device=dev)
+        f, n_it = rotating(lambda w4, st: bsq.w4a4_gemm(ap, asf, w4[0], w4[1], out, 1.0, 1.0, m, n, k, st), w4_list)
+        t = time_graph(torch, f, n_it)
+        hbm_row(f"a2_w4a4_gemm_small_m{m}", t, n * k // 2 + n * k // 16 + m * k // 2 + m * k // 16 + 2 * m * n,
+                {"tflops": round(2.0 * m * n * k / t / 1e12, 1), "l2": f"{len(w4_list)} rotating weight copies"})
+        del ap, asf, out
+    del w4_list
 
     # a3: row-wise FP8 quantiser (per-token activations of the FP8 projection)
     m, k = 8192, 5120

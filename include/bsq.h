@@ -102,7 +102,12 @@ BSQ_API bsq_status quantize_bf16_to_nvfp4(const uint16_t *in, uint8_t *packed,
  *   w_packed [n, k/2], w_scale [n, k/16]   weight (NVFP4)
  *   out      BF16 [m, n]
  *   C[i,j] = scaleA2 * scaleB2 * sum_k e2m1(A)e4m3(sfA) e2m1(W)e4m3(sfW)
- * FP32 accumulation in tensor memory, one BF16 rounding.
+ * FP32 accumulation in tensor memory, one BF16 rounding.  m <= 128 runs a
+ * kernel with the operands swapped (weight rows as the MMA's M operand),
+ * larger m one with 256 x 256 tiles on CTA pairs; the result is the same
+ * sum either way.  The kernel may begin its set-up while the previous kernel
+ * of the stream finishes (programmatic stream serialization); it reads its
+ * inputs only after that kernel has completed.
  * All pointers 16-byte aligned.
  * Errors: k % 16 != 0 -> INVALID_ARG; k % 256 != 0 -> UNSUPPORTED (the
  * scale rows must be 16-byte strided for the tensor-memory-access copies).

@@ -63,6 +63,11 @@ bsq_status w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint
     if (!a_packed || !a_scale || !w_packed || !w_scale || !out) return BSQ_ERR_INVALID_ARG;
     if (!al16(a_packed) || !al16(a_scale) || !al16(w_packed) || !al16(w_scale) || !al16(out))
         return BSQ_ERR_MISALIGNED;
+    // up to 128 activation rows the weight stream dominates: swapped
+    // operands, one CTA per 128 weight rows; above, CTA-pair 256 x 256 tiles
+    if (m <= 128)
+        return cuda_status(bsq::launch_w4a4_gemm_small(a_packed, a_scale, w_packed, w_scale, out, scaleA2 * scaleB2,
+                                                       m, n, k, cs(stream)));
     return cuda_status(
         bsq::launch_w4a4_gemm(a_packed, a_scale, w_packed, w_scale, out, scaleA2 * scaleB2, m, n, k, cs(stream)));
 }
@@ -194,7 +199,8 @@ uint64_t bsq_debug_launch_count(void) { return bsq::g_launches.load(std::memory_
 
 uint32_t bsq_debug_take_timeouts(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return 0xFFFFFFFFu;
-    return bsq::take_timeouts_gemm_w4a4() | bsq::take_timeouts_gemm_fp8() | bsq::take_timeouts_gemm_int8() |
+    return bsq::take_timeouts_gemm_w4a4() | bsq::take_timeouts_gemm_w4a4_small() | bsq::take_timeouts_gemm_fp8() |
+           bsq::take_timeouts_gemm_int8() |
            bsq::take_timeouts_gemv();
 }
 

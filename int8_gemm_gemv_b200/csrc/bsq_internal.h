@@ -14,6 +14,7 @@ void note_launch();
 // Per-file flags of bounded waits that ran out (read and cleared with a
 // device synchronisation; used by tests only).
 uint32_t take_timeouts_gemm_w4a4();
+uint32_t take_timeouts_gemm_w4a4_small();
 uint32_t take_timeouts_gemm_fp8();
 uint32_t take_timeouts_gemm_int8();
 uint32_t take_timeouts_gemv();
@@ -43,6 +44,10 @@ cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const
 cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
                              const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k,
                              cudaStream_t s);
+// M <= 128: swapped operands, one CTA per 128 weight rows (gemm_w4a4_small.cu)
+cudaError_t launch_w4a4_gemm_small(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
+                                   const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k,
+                                   cudaStream_t s);
 cudaError_t launch_fp8_gemm_rowscale(const uint8_t *a, const float *a_scale, const uint8_t *w,
                                      const float *w_scale, uint16_t *out, int m, int n, int k, cudaStream_t s);
 cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const float *a_scale,

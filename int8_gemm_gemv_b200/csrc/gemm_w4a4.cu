@@ -32,6 +32,10 @@
 // `w4a4_gemm_mfast` raster) and the working set stays in L2.  No load uses
 // cluster multicast.
 //
+// Launched with programmatic stream serialization: the set-up overlaps the
+// previous kernel of the stream, and the producer waits for it
+// (griddepcontrol.wait) before the first global load.
+//
 // Every mbarrier wait is bounded; on a timeout the kernel records it, stops
 // issuing work, drains what it issued, frees tensor memory and exits.
 #include <cstring>
@@ -137,6 +141,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tmB);
             prefetch_tensormap(&tmSFA);
             prefetch_tensormap(&tmSFB);
+            // everything above overlapped the previous kernel of the stream
+            // (programmatic stream serialization); global memory is read
+            // from here on, after it has completed.  Every other role's
+            // global access depends on these loads.
+            asm volatile("griddepcontrol.wait;" ::: "memory");
             uint32_t it = 0;
             bool ok = true;
             for (int t = pair; t < num_tiles && ok; t += npairs) {
@@ -393,7 +402,7 @@ cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, co
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
@@ -401,6 +410,11 @@ cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, co
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const int max_pairs = w4a4_max_pairs(cfg);
+    // the prologue (barriers, tensor memory, descriptor prefetch) may
+    // overlap the previous kernel, e.g. the activation quantiser's tail
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
     cfg.gridDim = dim3(2 * pairs);
     cudaError_t e = cudaLaunchKernelEx(&cfg, k_w4a4_gemm, tA, tB, tSA, tSB, tO, use_tma_store, out, scale_ab, m, n, k);

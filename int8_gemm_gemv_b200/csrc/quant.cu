@@ -224,6 +224,10 @@ __device__ __forceinline__ uint32_t nvfp4_codes_8(const uint4 &v, float d, const
 __global__ void __launch_bounds__(256) k_quant_nvfp4(const uint4 *__restrict__ in, uint2 *__restrict__ packed,
                                                      uint8_t *__restrict__ sf, float scale2, float t6,
                                                      int64_t nblocks) {
+    // a GEMM launched after this kernel with programmatic stream
+    // serialization may start its prologue now; it reads these outputs only
+    // after griddepcontrol.wait, i.e. after this grid has completed
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const Bracket t6b = bracket_of(t6);
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {

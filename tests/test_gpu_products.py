@@ -64,6 +64,26 @@ def test_w4a4_small_and_ragged(mnk):
     check_tol(g, ob, ab, f"w4a4 {mnk}")
 
 
+@pytest.mark.parametrize("m", [1, 2, 31, 32, 33, 64, 65, 100, 128])
+def test_w4a4_small_m_swapped(m):
+    """M <= 128 runs the swapped-operand kernel (weights as the MMA's M
+    operand, activations padded to 32, 64 or 128 columns); ragged N."""
+    n, k = 1984, 5120
+    args = nvfp4_from_oracle(m, n, k, seed=3)
+    g = run_w4a4(*args)
+    ob, _, ab = oracle.w4a4_gemm(*args)
+    check_tol(g, ob, ab, f"w4a4 small {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("mnk", [(4, 17408, 5120), (5, 1001, 512), (128, 130, 256), (3, 24, 768)])
+def test_w4a4_small_m_shapes(mnk):
+    m, n, k = mnk
+    args = nvfp4_from_oracle(m, n, k, seed=4)
+    g = run_w4a4(*args)
+    ob, _, ab = oracle.w4a4_gemm(*args)
+    check_tol(g, ob, ab, f"w4a4 small {mnk}")
+
+
 def test_w4a4_structured_one_hot():
     """One-hot activation rows pick single weight elements: checks nibble
     order, scale placement per row and per 16-block, and the M/N tiling."""
