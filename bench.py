@@ -274,20 +274,23 @@ def run_bsq(args, w, peaks, peak_src):
     barrier(dev)
     elapsed = t0.elapsed_time(t1) * 1e-3
     t_max = max_over_ranks(elapsed, dev)
-    # per-kernel durations: the same steps again, each kernel between its
-    # own events (this serialises the two kernels of a step)
-    ev = _events(torch, 3 * args.steps)
-    for i in range(args.steps):
-        j = i % nsets
-        wp, wsf, sb2 = w_codes[j]
-        ev[3 * i].record(stream)
-        bsq.quantize_bf16_to_nvfp4(a_dev[j], ap[j], asf[j], 1.0, m, k, stream)
-        ev[3 * i + 1].record(stream)
-        bsq.w4a4_gemm(ap[j], asf[j], wp, wsf, out, 1.0, sb2, m, n, k, stream)
-        ev[3 * i + 2].record(stream)
-    ev[-1].synchronize()
-    quant_t = statistics.mean(ev[3 * i].elapsed_time(ev[3 * i + 1]) for i in range(args.steps)) * 1e-3
-    gemm_t = statistics.mean(ev[3 * i + 1].elapsed_time(ev[3 * i + 2]) for i in range(args.steps)) * 1e-3
+    # per-kernel durations: each kernel of the step run alone, back to back
+    # over the same rotating input sets, between two events on the stream
+    def kernel_time(fn):
+        fn(0)
+        s0, s1 = _events(torch, 2)
+        s0.record(stream)
+        for i in range(args.steps):
+            fn(i)
+        s1.record(stream)
+        s1.synchronize()
+        return s0.elapsed_time(s1) * 1e-3 / args.steps
+
+    quant_t = kernel_time(lambda i: bsq.quantize_bf16_to_nvfp4(a_dev[i % nsets], ap[i % nsets], asf[i % nsets], 1.0,
+                                                               m, k, stream))
+    gemm_t = kernel_time(lambda i: bsq.w4a4_gemm(ap[i % nsets], asf[i % nsets], w_codes[i % nsets][0],
+                                                 w_codes[i % nsets][1], out, 1.0, w_codes[i % nsets][2], m, n, k,
+                                                 stream))
     flops = 2.0 * m * n * k
     value = world * flops * args.steps / t_max / 1e12
 
@@ -405,6 +408,25 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
             fn_of(inputs[it[0] % len(inputs)], st)
             it[0] += 1
         return f, reps_per_input * len(inputs)
+
+    # next row: block-scaled FP8 GEMV (w8a16_gemv_batch4 / _batch2), M = 1, 2, 4
+    n, k = 5120, 5120
+
+    def mk_bw():
+        wq = torch.empty((n, k), dtype=torch.uint8, device=dev)
+        S = torch.empty((n // 128, k // 128), dtype=torch.float32, device=dev)
+        bsq.quant_blockfp8(bf16_rand((n, k), 0.02), wq, S, n, k, stream)
+        return wq, S
+    bw_list = rotate(mk_bw, n * k)
+    for m in (1, 2, 4):
+        x = bf16_rand((m, k), 1.0)
+        out = torch.empty((m, n), dtype=torch.int16, device=dev)
+        f, n_it = rotating(lambda ws, st: bsq.fp8_gemv_blockscaled(x, ws[0], ws[1], out, m, n, k, st), bw_list)
+        t = time_graph(torch, f, n_it)
+        hbm_row(f"next_fp8_gemv_blockscaled_m{m}_n{n}_k{k}", t,
+                n * k + 4 * (n // 128) * (k // 128) + 2 * m * k + 2 * m * n,
+                {"l2": f"{len(bw_list)} rotating weight copies"})
+    del bw_list
 
     # a1: NVFP4 quantiser, 4096x5120 and 16384x5120 (inputs rotated past L2)
     for m in (4096, 16384):

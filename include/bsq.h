@@ -136,6 +136,25 @@ BSQ_API bsq_status fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w,
                              int m, int n, int k, bsq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * fp8_gemv_blockscaled -- fp8_gemv_batch.rs, `w8a16_gemv_batch4` and
+ * `w8a16_gemv_batch2` (the pages run them for m <= 4; here any 1 <= m <= 16).
+ *   in          BF16 [m, k]               (16-byte aligned)
+ *   w           E4M3 [n, k]               (16-byte aligned)
+ *   block_scale FP32 [n/128, k/128]       the block FP8 scale grid (4-byte
+ *                                          aligned), as quant_blockfp8 writes
+ *   out         BF16 [m, n]
+ *   out[i,j] = sum_k bf16(in[i,k]) * e4m3(w[j,k]) * block_scale[j/128, k/128]
+ * FP32 sums per 64-wide K chunk, scaled by their block and accumulated in
+ * FP32; one BF16 rounding.  As for fp8_gemv_rowscale, an output does not
+ * depend on m.
+ * Errors: m outside 1..16 or k % 16 != 0 -> INVALID_ARG; n or k not a
+ * multiple of 128 -> UNSUPPORTED (the block grid needs whole blocks).
+ * ---------------------------------------------------------------------- */
+BSQ_API bsq_status fp8_gemv_blockscaled(const uint16_t *in, const uint8_t *w,
+                             const float *block_scale, uint16_t *out,
+                             int m, int n, int k, bsq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * quant_rowwise_fp8 -- quantize_fns.rs, `quantize_to_fp8`, and
  * dispatch_proj_rowwise.rs, `quant_rowwise_fp8` (weights once, activations
  * per token).

@@ -16,7 +16,8 @@ import os
 __all__ = [
     "BsqError", "BSQ_OK", "BSQ_ERR_INVALID_ARG", "BSQ_ERR_MISALIGNED", "BSQ_ERR_UNSUPPORTED",
     "BSQ_ERR_CUDA", "BSQ_FP8_PER_ROW", "BSQ_FP8_BLOCK_SCALED", "BSQ_FP8_SINGLE_SCALE", "BSQ_BF16",
-    "BSQ_NVFP4", "quantize_bf16_to_nvfp4", "w4a4_gemm", "fp8_gemv_rowscale", "quant_rowwise_fp8",
+    "BSQ_NVFP4", "quantize_bf16_to_nvfp4", "w4a4_gemm", "fp8_gemv_rowscale", "fp8_gemv_blockscaled",
+    "quant_rowwise_fp8",
     "quant_blockfp8", "requant_w_nvfp4_int8", "quant_act_int8_per32", "int8_blockscaled_gemm",
     "int8_w4a8_prefill", "int8_w4a8_prefill_noalloc", "requant_blockfp8_to_rowwise", "fp8_gemm_rowscale", "bsq_amax_bf16",
     "status_string", "debug_launch_count", "debug_take_timeouts", "library_path", "lib",
@@ -47,6 +48,7 @@ _SIGS = {
     "quantize_bf16_to_nvfp4": [_P, _P, _P, _F, _I, _I, _P],
     "w4a4_gemm": [_P, _P, _P, _P, _P, _F, _F, _I, _I, _I, _P],
     "fp8_gemv_rowscale": [_P, _P, _P, _P, _I, _I, _I, _P],
+    "fp8_gemv_blockscaled": [_P, _P, _P, _P, _I, _I, _I, _P],
     "quant_rowwise_fp8": [_P, _P, _P, _I, _I, _P],
     "quant_blockfp8": [_P, _P, _P, _I, _I, _P],
     "requant_w_nvfp4_int8": [_P, _P, _F, _P, _P, _I, _I, _P],
@@ -133,6 +135,10 @@ def w4a4_gemm(a_packed, a_scale, w_packed, w_scale, out, scaleA2, scaleB2, m, n,
 
 def fp8_gemv_rowscale(inp, w, row_scale, out, m, n, k, stream=None):
     _call("fp8_gemv_rowscale", _ptr(inp), _ptr(w), _ptr(row_scale), _ptr(out), m, n, k, _stream(stream))
+
+
+def fp8_gemv_blockscaled(inp, w, block_scale, out, m, n, k, stream=None):
+    _call("fp8_gemv_blockscaled", _ptr(inp), _ptr(w), _ptr(block_scale), _ptr(out), m, n, k, _stream(stream))
 
 
 def quant_rowwise_fp8(inp, q, scale, rows, k, stream=None):

@@ -82,6 +82,17 @@ bsq_status fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *
     return cuda_status(bsq::launch_fp8_gemv_rowscale(in, w, row_scale, out, m, n, k, cs(stream)));
 }
 
+bsq_status fp8_gemv_blockscaled(const uint16_t *in, const uint8_t *w, const float *block_scale, uint16_t *out,
+                                int m, int n, int k, bsq_stream_t stream) {
+    if (m < 1 || m > 16 || n < 0 || k <= 0 || k % 16) return BSQ_ERR_INVALID_ARG;
+    if (n % 128 || k % 128) return BSQ_ERR_UNSUPPORTED;
+    if (n == 0) return BSQ_OK;
+    if (!in || !w || !block_scale || !out) return BSQ_ERR_INVALID_ARG;
+    if (!al16(in) || !al16(w) || !al4(block_scale) || (reinterpret_cast<uintptr_t>(out) & 1u))
+        return BSQ_ERR_MISALIGNED;
+    return cuda_status(bsq::launch_fp8_gemv_blockscaled(in, w, block_scale, out, m, n, k, cs(stream)));
+}
+
 bsq_status quant_rowwise_fp8(const uint16_t *in, uint8_t *q, float *scale, int rows, int k, bsq_stream_t stream) {
     if (rows < 0 || k <= 0 || k % 16) return BSQ_ERR_INVALID_ARG;
     if (rows == 0) return BSQ_OK;

@@ -39,6 +39,8 @@ cudaError_t launch_amax_bf16(const uint16_t *x, size_t count, float *amax, cudaS
 // ---- launchers (gemv_fp8.cu) ----
 cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *row_scale, uint16_t *out,
                                      int m, int n, int k, cudaStream_t s);
+cudaError_t launch_fp8_gemv_blockscaled(const uint16_t *in, const uint8_t *w, const float *block_scale,
+                                        uint16_t *out, int m, int n, int k, cudaStream_t s);
 
 // ---- launchers (gemm_*.cu) ----
 cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,

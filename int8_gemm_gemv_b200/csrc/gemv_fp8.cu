@@ -2,6 +2,11 @@
 // `fp8_gemv_rowscale_batch8_rt2`, `fp8_gemv_rowscale_batch16_rt2`,
 // `dense_gemv_fp8w_batch2`):
 //   out[m, n] = row_scale[n] * sum_k bf16(in[m, k]) * e4m3(W[n, k])
+// and its block-scaled sibling (`w8a16_gemv_batch4`, `w8a16_gemv_batch2`):
+//   out[m, n] = sum_k bf16(in[m, k]) * e4m3(W[n, k]) * S[n / 128, k / 128]
+// where each warp's 64-byte K chunk of a stage lies in one 128-wide scale
+// block, so its MMAs for the stage go into a zeroed accumulator that is
+// then added to the running sum times the scale of the row's block.
 //
 // The weight stream (N*K bytes, read once) is the whole cost.  Design:
 //   * persistent: one CTA per SM, each owning a contiguous range of 8-row
@@ -109,7 +114,7 @@ __device__ __forceinline__ uint32_t stage_offset(int u, int w, int r, int t) {
     return (uint32_t)(u * TILE_BYTES + box * (16 * BOX) + r * BOX + ((unit ^ (r & 7)) << 4));
 }
 
-template <int MT>
+template <int MT, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
     k_fp8_gemv(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW8,
                const uint8_t *__restrict__ wptr, const uint16_t *__restrict__ X, const float *__restrict__ row_scale,
@@ -228,6 +233,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = it % STAGES;
             const int kk = q * KS;  // + 64 * warp + 16 * t, folded into x0/x1
             const bool kok = kk + 64 * warp + 16 * t < K;
+            // block scales of this warp's chunk for rows g and g + 8 of each
+            // tile (row_scale is the [N/128, K/128] grid here)
+            float bs[2][2];
+            if (BS) {
+                const int kbn = K >> 7;
+                const int kbi = min((kk + 64 * warp) >> 7, kbn - 1);
+#pragma unroll
+                for (int u = 0; u < 2; u++) {
+                    const int r0 = min(row_begin + (t0 + u) * 16 + g, N - 1);
+                    const int r1 = min(r0 + 8, N - 1);
+                    bs[u][0] = __ldg(row_scale + (int64_t)(r0 >> 7) * kbn + kbi);
+                    bs[u][1] = __ldg(row_scale + (int64_t)(r1 >> 7) * kbn + kbi);
+                }
+            }
             // activation fragments for this chunk (shared by both tiles)
             uint4 xa[2], xb[2];
             xa[0] = (okX0 && kok) ? ld_x_v4(x0 + kk) : z;
@@ -261,6 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (u == 1 && nt < 2) break;
                 const uint32_t a_w[4] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w};
                 const uint32_t b_w[4] = {wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+                // block-scaled: this chunk's sums first, then scaled into acc
+                float d[MT][4];
+#pragma unroll
+                for (int i = 0; i < MT; i++) d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.0f;
+                float(&dst)[MT][4] = BS ? d : acc[u];
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     uint32_t a[4];
@@ -268,8 +292,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     a[1] = e4m3x2_to_bf16x2(b_w[j] & 0xFFFF);  // row g+8, k 4j, 4j+1
                     a[2] = e4m3x2_to_bf16x2(a_w[j] >> 16);     // row g,   k 4j+2, 4j+3
                     a[3] = e4m3x2_to_bf16x2(b_w[j] >> 16);     // row g+8, k 4j+2, 4j+3
-                    mma_bf16_16816(acc[u][0], a, xa_w[2 * j], xa_w[2 * j + 1]);
-                    if (MT == 2) mma_bf16_16816(acc[u][MT - 1], a, xb_w[2 * j], xb_w[2 * j + 1]);
+                    mma_bf16_16816(dst[0], a, xa_w[2 * j], xa_w[2 * j + 1]);
+                    if (MT == 2) mma_bf16_16816(dst[MT - 1], a, xb_w[2 * j], xb_w[2 * j + 1]);
+                }
+                if (BS) {
+                    // d[i][0..1]: row g; d[i][2..3]: row g + 8
+#pragma unroll
+                    for (int i = 0; i < MT; i++) {
+                        acc[u][i][0] = __fmaf_rn(d[i][0], bs[u][0], acc[u][i][0]);
+                        acc[u][i][1] = __fmaf_rn(d[i][1], bs[u][0], acc[u][i][1]);
+                        acc[u][i][2] = __fmaf_rn(d[i][2], bs[u][1], acc[u][i][2]);
+                        acc[u][i][3] = __fmaf_rn(d[i][3], bs[u][1], acc[u][i][3]);
+                    }
                 }
             }
         }
@@ -294,7 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n = row_begin + (t0 + u) * 16 + g + 8 * (r >> 1);
                 const int m = 8 * i + 2 * t + (r & 1);
                 if (n < row_end && m < M)
-                    out[(int64_t)m * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v[r] * __ldg(row_scale + n)));
+                    out[(int64_t)m * N + n] =
+                        __bfloat16_as_ushort(__float2bfloat16_rn(BS ? v[r] : v[r] * __ldg(row_scale + n)));
             }
         }
         consumers_sync();
@@ -311,7 +346,7 @@ uint32_t take_timeouts_gemv() {
     return v;
 }
 
-template <int MT>
+template <int MT, bool BS>
 static cudaError_t launch_mt(const CUtensorMap &tm, const CUtensorMap &tm8, int tm3d, const uint8_t *w,
                              const uint16_t *in, const float *row_scale, uint16_t *out, int m, int n, int k,
                              cudaStream_t s) {
@@ -319,7 +354,7 @@ static cudaError_t launch_mt(const CUtensorMap &tm, const CUtensorMap &tm8, int 
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_fp8_gemv<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(k_fp8_gemv<MT, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem_bytes<MT>());
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
@@ -336,11 +371,12 @@ static cudaError_t launch_mt(const CUtensorMap &tm, const CUtensorMap &tm8, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_fp8_gemv<MT>, tm, tm8, w, in, row_scale, out, m, n, k, tm3d);
+    return cudaLaunchKernelEx(&cfg, k_fp8_gemv<MT, BS>, tm, tm8, w, in, row_scale, out, m, n, k, tm3d);
 }
 
-cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *row_scale, uint16_t *out,
-                                     int m, int n, int k, cudaStream_t s) {
+template <bool BS>
+static cudaError_t launch_gemv(const uint16_t *in, const uint8_t *w, const float *scale, uint16_t *out, int m, int n,
+                               int k, cudaStream_t s) {
     alignas(64) CUtensorMap tm, tm8;
     // K a multiple of 128: one 16 KB copy per tile and stage; otherwise eight
     // 2 KB copies (the last chunk of a row may be partial).  8-row tiles:
@@ -350,10 +386,20 @@ cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const
                           : make_tmap_2d(&tm, w, 1, k, n, k, BOX, 16, true, false)) &&
                     make_tmap_2d(&tm8, w, 1, k, n, k, BOX, 8, true, false);
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = m <= 8 ? launch_mt<1>(tm, tm8, tm3d, w, in, row_scale, out, m, n, k, s)
-                           : launch_mt<2>(tm, tm8, tm3d, w, in, row_scale, out, m, n, k, s);
+    cudaError_t e = m <= 8 ? launch_mt<1, BS>(tm, tm8, tm3d, w, in, scale, out, m, n, k, s)
+                           : launch_mt<2, BS>(tm, tm8, tm3d, w, in, scale, out, m, n, k, s);
     note_launch();
     return e;
+}
+
+cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *row_scale, uint16_t *out,
+                                     int m, int n, int k, cudaStream_t s) {
+    return launch_gemv<false>(in, w, row_scale, out, m, n, k, s);
+}
+
+cudaError_t launch_fp8_gemv_blockscaled(const uint16_t *in, const uint8_t *w, const float *block_scale,
+                                        uint16_t *out, int m, int n, int k, cudaStream_t s) {
+    return launch_gemv<true>(in, w, block_scale, out, m, n, k, s);
 }
 
 }  // namespace bsq

@@ -3,9 +3,9 @@
     python -m int8_gemm_gemv_b200.profile_case w4a4 --m 4096 --n 17408 --k 5120 --iters 3
 
 Inputs are random codes in device memory (the kernel's cost does not depend
-on their values beyond power); nothing is checked.  Kinds: w4a4, fp8gemm,
-int8gemm, gemv, quant_nvfp4, quant_rowfp8, quant_int8, requant_w,
-requant_block.
+on their values beyond power); nothing is checked.  Kinds: w4a4 (M <= 128
+runs the few-row kernel), fp8gemm, int8gemm, gemv, gemv_bs (block-scaled),
+quant_nvfp4, quant_rowfp8, quant_int8, requant_w, requant_block.
 """
 from __future__ import annotations
 
@@ -35,7 +35,8 @@ def main():
     def bf16(shape, std=1.0):
         return (torch.randn(shape, device=dev, generator=g) * std).to(torch.bfloat16)
 
-    out = torch.empty((m, n), dtype=torch.int16, device=dev) if a.kind in ("w4a4", "fp8gemm", "int8gemm", "gemv") else None
+    out = torch.empty((m, n), dtype=torch.int16, device=dev) if a.kind in ("w4a4", "fp8gemm", "int8gemm", "gemv",
+                                                                          "gemv_bs") else None
     if a.kind == "w4a4":
         ap, asf, wp, wsf = u8((m, k // 2)), u8((m, k // 16), 0x30, 0x40), u8((n, k // 2)), u8((n, k // 16), 0x30, 0x40)
         fn = lambda: bsq.w4a4_gemm(ap, asf, wp, wsf, out, 1.0, 1.0, m, n, k)
@@ -48,6 +49,10 @@ def main():
         w = torch.randint(-127, 128, (n, k), dtype=torch.int8, device=dev)
         sa, sw = torch.rand(m, k // 32, device=dev), torch.rand(n, k // 32, device=dev)
         fn = lambda: bsq.int8_blockscaled_gemm(x, w, sa, sw, out, m, n, k)
+    elif a.kind == "gemv_bs":
+        x, w = bf16((m, k)), u8((n, k), 0, 0x7F)
+        S = torch.rand(n // 128, k // 128, device=dev)
+        fn = lambda: bsq.fp8_gemv_blockscaled(x, w, S, out, m, n, k)
     elif a.kind == "gemv":
         x, w, s = bf16((m, k)), u8((n, k), 0, 0x7F), torch.rand(n, device=dev)
         fn = lambda: bsq.fp8_gemv_rowscale(x, w, s, out, m, n, k)

@@ -75,6 +75,7 @@ def _declare(L):
     prod_tail = [_i64, _i64, _i64, _i64p, _i64, _u16p, _f64p, _f64p]
     L.or_w4a4_gemm.argtypes = [_u8p, _u8p, _u8p, _u8p, ctypes.c_float, ctypes.c_float] + prod_tail
     L.or_fp8_gemv_rowscale.argtypes = [_u16p, _u8p, _f32p] + prod_tail
+    L.or_fp8_gemv_blockscaled.argtypes = [_u16p, _u8p, _f32p] + prod_tail
     L.or_int8_blockscaled_gemm.argtypes = [_i8p, _i8p, _f32p, _f32p] + prod_tail
     L.or_fp8_gemm_rowscale.argtypes = [_u8p, _f32p, _u8p, _f32p] + prod_tail
 
@@ -219,6 +220,20 @@ def fp8_gemv_rowscale(inp_bf16, w, row_scale, rows=None):
     lib().or_fp8_gemv_rowscale(_p(inp, _u16p), _p(w, _u8p), _p(row_scale, _f32p),
                                m, n, k, _p(r, _i64p), nr,
                                _p(ob, _u16p), _p(oe, _f64p), _p(oa, _f64p))
+    return ob, oe, oa
+
+
+def fp8_gemv_blockscaled(inp_bf16, w, block_scale, rows=None):
+    """Block-scaled FP8 GEMV: block_scale is the FP32 grid [N/128, K/128]."""
+    inp, w = _c(inp_bf16, np.uint16), _c(w, np.uint8)
+    block_scale = _c(block_scale, np.float32)
+    m, k = inp.shape
+    n = w.shape[0]
+    assert n % 128 == 0 and k % 128 == 0 and block_scale.shape == (n // 128, k // 128)
+    r, nr, ob, oe, oa = _prod_out(rows, m, n)
+    lib().or_fp8_gemv_blockscaled(_p(inp, _u16p), _p(w, _u8p), _p(block_scale, _f32p),
+                                  m, n, k, _p(r, _i64p), nr,
+                                  _p(ob, _u16p), _p(oe, _f64p), _p(oa, _f64p))
     return ob, oe, oa
 
 

@@ -387,6 +387,33 @@ void or_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w,
     }
 }
 
+/* Block-scaled FP8 GEMV (fp8_gemv_batch.rs, `w8a16_gemv_batch4` doc
+ * comment): every product carries the scale of the 128 x 128 weight block
+ * it falls in; the sum is exact in double, rounded once to BF16.           */
+void or_fp8_gemv_blockscaled(const uint16_t *in, const uint8_t *w,
+                             const float *block_scale,
+                             int64_t m, int64_t n, int64_t k,
+                             const int64_t *rows, int64_t nrows,
+                             uint16_t *out_bf16, double *out_exact, double *abssum) {
+    if (!e4m3_ready) e4m3_build();
+    if (!rows) nrows = m;
+    const int64_t kb = k / 128;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; i++) {
+        int64_t r = rows ? rows[i] : i;
+        for (int64_t j = 0; j < n; j++) {
+            double acc = 0.0, abs_acc = 0.0;
+            for (int64_t e = 0; e < k; e++) {
+                double sc = (double)block_scale[(j / 128) * kb + e / 128];
+                double p = (double)or_bf16_value(in[r * k + e]) * E4M3_TAB[w[j * k + e]] * sc;
+                acc += p;
+                abs_acc += fabs(p);
+            }
+            store_out(i, n, j, acc, abs_acc, out_bf16, out_exact, abssum);
+        }
+    }
+}
+
 /* int8 block-scaled GEMM (gemm_dense_int8.rs, `int8_gemm_faith2_prefill`
  * step (b)): for every 32-block b the int32 partial sum of a*w is exact, then
  *   C[m,n] = sum_b partial_b * sA[m,b] * sW[n,b]                           */

@@ -74,6 +74,16 @@ void or_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w,
                           int64_t m, int64_t n, int64_t k,
                           const int64_t *rows, int64_t nrows,
                           uint16_t *out_bf16, double *out_exact, double *abssum);
+/* Block-scaled FP8 GEMV (fp8_gemv_batch.rs, `w8a16_gemv_batch4` and
+ * `w8a16_gemv_batch2` doc comments: BF16 input [M, K], E4M3 weight with the
+ * 2-D block scales of the block FP8 format, BF16 output [M, N]):
+ *   out[m, n] = sum_k bf16(in[m, k]) * e4m3(W[n, k]) * S[n / 128, k / 128]
+ * with S the FP32 grid [N/128, K/128] (N, K multiples of 128).            */
+void or_fp8_gemv_blockscaled(const uint16_t *in, const uint8_t *w,
+                             const float *block_scale,
+                             int64_t m, int64_t n, int64_t k,
+                             const int64_t *rows, int64_t nrows,
+                             uint16_t *out_bf16, double *out_exact, double *abssum);
 void or_int8_blockscaled_gemm(const int8_t *a, const int8_t *w,
                               const float *a_scale, const float *w_scale,
                               int64_t m, int64_t n, int64_t k,

@@ -74,6 +74,12 @@ def test_validation_launches_nothing():
         (1, "fp8_gemv_rowscale", (A16, A16b, A16c, A16d, 8, 64, 72, 0)),         # k % 16
         (2, "fp8_gemv_rowscale", (A16, ODD, A16c, A16d, 8, 64, 64, 0)),
         (0, "fp8_gemv_rowscale", (A16, A16b, A16c, A16d, 8, 0, 64, 0)),
+        (1, "fp8_gemv_blockscaled", (A16, A16b, A16c, A16d, 0, 128, 128, 0)),   # m = 0
+        (1, "fp8_gemv_blockscaled", (A16, A16b, A16c, A16d, 4, 128, 120, 0)),   # k % 16
+        (3, "fp8_gemv_blockscaled", (A16, A16b, A16c, A16d, 4, 100, 128, 0)),   # n % 128
+        (3, "fp8_gemv_blockscaled", (A16, A16b, A16c, A16d, 4, 128, 144, 0)),   # k % 128
+        (2, "fp8_gemv_blockscaled", (A16, A16b, A16c, ODD, 4, 128, 128, 0)),    # out odd
+        (0, "fp8_gemv_blockscaled", (A16, A16b, A16c, A16d, 4, 0, 128, 0)),
         (1, "quant_rowwise_fp8", (A16, A16b, A16c, 4, 40, 0)),
         (1, "quant_blockfp8", (A16, A16b, A16c, 100, 128, 0)),
         (1, "requant_w_nvfp4_int8", (A16, A16b, 1.0, A16c, A16d, 4, 48, 0)),

@@ -171,6 +171,36 @@ def test_gemv_ragged(nk):
         check_tol(g, ob, ab, f"gemv {m}x{n}x{k}")
 
 
+def run_gemv_bs(inp, wq, S):
+    m, k = inp.shape
+    n = wq.shape[0]
+    out = bf16_out((m, n))
+    bsq.fp8_gemv_blockscaled(to_dev(inp), to_dev(wq), to_dev(S), out, m, n, k)
+    torch.cuda.synchronize()
+    return host(out, np.uint16)
+
+
+@pytest.mark.parametrize("mnk", [(1, 5120, 5120), (2, 5120, 5120), (4, 5120, 5120), (16, 1024, 1024),
+                                 (3, 256, 128), (9, 1152, 1920), (2, 8192, 5120)])
+def test_gemv_blockscaled(mnk):
+    """Block-scaled FP8 weights (the block FP8 format, per-128x128 scales)."""
+    m, n, k = mnk
+    inp, w_bf = synth.gemv_inputs(m, n, k, seed=5)
+    wq, S = oracle.quant_blockfp8(w_bf)
+    g = run_gemv_bs(inp, wq, S)
+    ob, _, ab = oracle.fp8_gemv_blockscaled(inp, wq, S)
+    check_tol(g, ob, ab, f"gemv block-scaled {mnk}")
+
+
+def test_gemv_blockscaled_row_independent_of_batch():
+    inp, w_bf = synth.gemv_inputs(16, 1024, 2048, seed=6)
+    wq, S = oracle.quant_blockfp8(w_bf)
+    all16 = run_gemv_bs(inp, wq, S)
+    for m in (1, 4):
+        part = run_gemv_bs(inp[:m].copy(), wq, S)
+        assert np.array_equal(part, all16[:m])
+
+
 def test_gemv_lm_head_shape():
     n, k = 151936, 5120
     wq = synth.uniform_bytes((n, k), 0, 21, 0, 0x7F) | (synth.uniform_bytes((n, k), 0, 22, 0, 2) << 7)

@@ -525,6 +525,45 @@ def test_fp8_gemv_matches_float64_and_identity():
     assert np.array_equal(ob1[0], ob16[3])
 
 
+def _e4m3_tab():
+    return np.array([oracle.e4m3_value(c) for c in range(256)])
+
+
+def test_fp8_gemv_blockscaled_matches_float64_blocks():
+    """Block scales: each 128 x 128 weight block's products carry that
+    block's scale (fp8_gemv_batch.rs, `w8a16_gemv_batch4`).  Checked against
+    an independent float64 sum built block by block, with distinct scales
+    per row block and per K block, so a swapped or dropped index fails."""
+    m, n, k = 3, 256, 384
+    inp = synth.normal_bf16((m, k), 1.0, 0, 21)
+    w = synth.uniform_bytes((n, k), 21, 2, 0x00, 0x7F)  # finite E4M3 codes
+    S = np.array([[0.5, 2.0, 0.125], [3.0, 0.25, 1.5]], np.float32)
+    ob, ex, ab = oracle.fp8_gemv_blockscaled(inp, w, S)
+    x = (inp.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    wv = _e4m3_tab()[w]
+    ref = np.zeros((m, n))
+    for nb in range(2):
+        for kb in range(3):
+            ref[:, nb * 128:(nb + 1) * 128] += S[nb, kb] * (
+                x[:, kb * 128:(kb + 1) * 128] @ wv[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128].T)
+    assert np.allclose(ex, ref, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(ob, np.array([[oracle.bf16_encode(v) for v in row] for row in ref], np.uint16))
+    assert np.all(ab >= np.abs(ex) - 1e-9)
+
+
+def test_fp8_gemv_blockscaled_uniform_scale_is_rowscale():
+    """With one scale per 128-row block and no change along K, the block
+    form reduces to the row-scaled GEMV with those row scales."""
+    m, n, k = 2, 256, 256
+    inp = synth.normal_bf16((m, k), 1.0, 0, 22)
+    w = synth.uniform_bytes((n, k), 22, 2, 0x00, 0x7F)
+    S = np.array([[0.75, 0.75], [4.0, 4.0]], np.float32)
+    _, ex_b, _ = oracle.fp8_gemv_blockscaled(inp, w, S)
+    rs = np.repeat(S[:, 0], 128).astype(np.float32)
+    _, ex_r, _ = oracle.fp8_gemv_rowscale(inp, w, rs)
+    assert np.allclose(ex_b, ex_r, rtol=1e-12, atol=1e-12)
+
+
 def test_int8_gemm_matches_integer_blocks():
     g = np.random.default_rng(33)
     a = g.integers(-127, 128, size=(6, 128)).astype(np.int8)
