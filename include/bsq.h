@@ -97,6 +97,25 @@ BSQ_API bsq_status quantize_bf16_to_nvfp4(const uint16_t *in, uint8_t *packed,
                                   bsq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * quantize_bf16_to_nvfp4_devscale -- quantize_bf16_to_nvfp4 with the
+ * per-tensor scale2 formed on the device from the tensor's amax (the weight
+ * rule of gemm_fp4.rs: scale2 = amax / (6 * 448)), so a weight can be
+ * quantised without a round trip through the host.
+ *   amax       FP32 [1] device, e.g. from bsq_amax_bf16 (4-byte aligned)
+ *   scale2_out FP32 [1] device or NULL: receives scale2, for
+ *              w4a4_gemm_devscale (4-byte aligned)
+ *   The kernel computes scale2 = amax / 2688 and t = 6 * scale2 with the
+ *   same FP32 round-to-nearest steps as the host form, so its codes and
+ *   scales equal those of quantize_bf16_to_nvfp4 given that scale2.  An
+ *   all-zero tensor (amax = 0) gets scale codes 0 and codes +0/-0.
+ * Errors: as quantize_bf16_to_nvfp4; amax NULL -> INVALID_ARG.
+ * ---------------------------------------------------------------------- */
+BSQ_API bsq_status quantize_bf16_to_nvfp4_devscale(const uint16_t *in, uint8_t *packed,
+                                  uint8_t *scale, const float *amax,
+                                  float *scale2_out, int m, int k,
+                                  bsq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * w4a4_gemm -- gemm_fp4.rs, `w4a4_gemm` (NVFP4 x NVFP4 on FP4 tensor cores).
  *   a_packed [m, k/2], a_scale [m, k/16]   activations (NVFP4)
  *   w_packed [n, k/2], w_scale [n, k/16]   weight (NVFP4)
@@ -115,6 +134,19 @@ BSQ_API bsq_status quantize_bf16_to_nvfp4(const uint16_t *in, uint8_t *packed,
 BSQ_API bsq_status w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale,
                      const uint8_t *w_packed, const uint8_t *w_scale,
                      uint16_t *out, float scaleA2, float scaleB2,
+                     int m, int n, int k, bsq_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * w4a4_gemm_devscale -- w4a4_gemm with the weight's scale2 read from device
+ * memory (scaleB2 -> FP32 [1] device, 4-byte aligned, e.g. the scale2_out
+ * of quantize_bf16_to_nvfp4_devscale).  The kernel multiplies scaleA2 by
+ * it in FP32 (as the host form multiplies the two floats) after the
+ * previous kernel of the stream has completed.
+ * Errors: as w4a4_gemm; scaleB2 NULL with m, n > 0 -> INVALID_ARG.
+ * ---------------------------------------------------------------------- */
+BSQ_API bsq_status w4a4_gemm_devscale(const uint8_t *a_packed, const uint8_t *a_scale,
+                     const uint8_t *w_packed, const uint8_t *w_scale,
+                     uint16_t *out, float scaleA2, const float *scaleB2,
                      int m, int n, int k, bsq_stream_t stream);
 
 /* ------------------------------------------------------------------------

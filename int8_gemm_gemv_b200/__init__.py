@@ -16,7 +16,8 @@ import os
 __all__ = [
     "BsqError", "BSQ_OK", "BSQ_ERR_INVALID_ARG", "BSQ_ERR_MISALIGNED", "BSQ_ERR_UNSUPPORTED",
     "BSQ_ERR_CUDA", "BSQ_FP8_PER_ROW", "BSQ_FP8_BLOCK_SCALED", "BSQ_FP8_SINGLE_SCALE", "BSQ_BF16",
-    "BSQ_NVFP4", "quantize_bf16_to_nvfp4", "w4a4_gemm", "fp8_gemv_rowscale", "fp8_gemv_blockscaled",
+    "BSQ_NVFP4", "quantize_bf16_to_nvfp4", "quantize_bf16_to_nvfp4_devscale", "w4a4_gemm",
+    "w4a4_gemm_devscale", "fp8_gemv_rowscale", "fp8_gemv_blockscaled",
     "quant_rowwise_fp8",
     "quant_blockfp8", "requant_w_nvfp4_int8", "quant_act_int8_per32", "int8_blockscaled_gemm",
     "int8_w4a8_prefill", "int8_w4a8_prefill_noalloc", "requant_blockfp8_to_rowwise", "fp8_gemm_rowscale", "bsq_amax_bf16",
@@ -46,7 +47,9 @@ _F = ctypes.c_float
 
 _SIGS = {
     "quantize_bf16_to_nvfp4": [_P, _P, _P, _F, _I, _I, _P],
+    "quantize_bf16_to_nvfp4_devscale": [_P, _P, _P, _P, _P, _I, _I, _P],
     "w4a4_gemm": [_P, _P, _P, _P, _P, _F, _F, _I, _I, _I, _P],
+    "w4a4_gemm_devscale": [_P, _P, _P, _P, _P, _F, _P, _I, _I, _I, _P],
     "fp8_gemv_rowscale": [_P, _P, _P, _P, _I, _I, _I, _P],
     "fp8_gemv_blockscaled": [_P, _P, _P, _P, _I, _I, _I, _P],
     "quant_rowwise_fp8": [_P, _P, _P, _I, _I, _P],
@@ -126,6 +129,17 @@ def debug_take_timeouts() -> int:
 
 def quantize_bf16_to_nvfp4(inp, packed, scale, scale2, m, k, stream=None):
     _call("quantize_bf16_to_nvfp4", _ptr(inp), _ptr(packed), _ptr(scale), scale2, m, k, _stream(stream))
+
+
+def quantize_bf16_to_nvfp4_devscale(inp, packed, scale, amax, scale2_out, m, k, stream=None):
+    """scale2 = amax / (6 * 448) formed on the device; scale2_out may be None."""
+    _call("quantize_bf16_to_nvfp4_devscale", _ptr(inp), _ptr(packed), _ptr(scale), _ptr(amax), _ptr(scale2_out),
+          m, k, _stream(stream))
+
+
+def w4a4_gemm_devscale(a_packed, a_scale, w_packed, w_scale, out, scaleA2, scaleB2_dev, m, n, k, stream=None):
+    _call("w4a4_gemm_devscale", _ptr(a_packed), _ptr(a_scale), _ptr(w_packed), _ptr(w_scale), _ptr(out),
+          scaleA2, _ptr(scaleB2_dev), m, n, k, _stream(stream))
 
 
 def w4a4_gemm(a_packed, a_scale, w_packed, w_scale, out, scaleA2, scaleB2, m, n, k, stream=None):

@@ -50,14 +50,23 @@ bsq_status quantize_bf16_to_nvfp4(const uint16_t *in, uint8_t *packed, uint8_t *
     if (m == 0) return BSQ_OK;
     if (!in || !packed || !scale) return BSQ_ERR_INVALID_ARG;
     if (!al16(in) || !al16(packed)) return BSQ_ERR_MISALIGNED;
-    return cuda_status(bsq::launch_quant_nvfp4(in, packed, scale, scale2, m, k, cs(stream)));
+    return cuda_status(bsq::launch_quant_nvfp4(in, packed, scale, scale2, nullptr, nullptr, m, k, cs(stream)));
 }
 
-bsq_status w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
-                     const uint8_t *w_scale, uint16_t *out, float scaleA2, float scaleB2, int m, int n, int k,
-                     bsq_stream_t stream) {
-    if (m < 0 || n < 0 || k <= 0 || k % 16 || !std::isfinite(scaleA2) || !std::isfinite(scaleB2))
-        return BSQ_ERR_INVALID_ARG;
+bsq_status quantize_bf16_to_nvfp4_devscale(const uint16_t *in, uint8_t *packed, uint8_t *scale, const float *amax,
+                                           float *scale2_out, int m, int k, bsq_stream_t stream) {
+    if (m < 0 || k <= 0 || k % 16) return BSQ_ERR_INVALID_ARG;
+    if (m == 0) return BSQ_OK;
+    if (!in || !packed || !scale || !amax) return BSQ_ERR_INVALID_ARG;
+    if (!al16(in) || !al16(packed) || !al4(amax) || (scale2_out && !al4(scale2_out))) return BSQ_ERR_MISALIGNED;
+    return cuda_status(bsq::launch_quant_nvfp4(in, packed, scale, 0.0f, amax, scale2_out, m, k, cs(stream)));
+}
+
+namespace {
+
+bsq_status w4a4_common(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
+                       const uint8_t *w_scale, uint16_t *out, float scale_ab, const float *scale_b_dev, int m, int n,
+                       int k, bsq_stream_t stream) {
     if (k % 256) return BSQ_ERR_UNSUPPORTED;
     if (m == 0 || n == 0) return BSQ_OK;
     if (!a_packed || !a_scale || !w_packed || !w_scale || !out) return BSQ_ERR_INVALID_ARG;
@@ -66,10 +75,29 @@ bsq_status w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint
     // up to 128 activation rows the weight stream dominates: swapped
     // operands, one CTA per 128 weight rows; above, CTA-pair 256 x 256 tiles
     if (m <= 128)
-        return cuda_status(bsq::launch_w4a4_gemm_small(a_packed, a_scale, w_packed, w_scale, out, scaleA2 * scaleB2,
-                                                       m, n, k, cs(stream)));
-    return cuda_status(
-        bsq::launch_w4a4_gemm(a_packed, a_scale, w_packed, w_scale, out, scaleA2 * scaleB2, m, n, k, cs(stream)));
+        return cuda_status(bsq::launch_w4a4_gemm_small(a_packed, a_scale, w_packed, w_scale, out, scale_ab,
+                                                       scale_b_dev, m, n, k, cs(stream)));
+    return cuda_status(bsq::launch_w4a4_gemm(a_packed, a_scale, w_packed, w_scale, out, scale_ab, scale_b_dev, m, n,
+                                             k, cs(stream)));
+}
+
+}  // namespace
+
+bsq_status w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
+                     const uint8_t *w_scale, uint16_t *out, float scaleA2, float scaleB2, int m, int n, int k,
+                     bsq_stream_t stream) {
+    if (m < 0 || n < 0 || k <= 0 || k % 16 || !std::isfinite(scaleA2) || !std::isfinite(scaleB2))
+        return BSQ_ERR_INVALID_ARG;
+    return w4a4_common(a_packed, a_scale, w_packed, w_scale, out, scaleA2 * scaleB2, nullptr, m, n, k, stream);
+}
+
+bsq_status w4a4_gemm_devscale(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
+                              const uint8_t *w_scale, uint16_t *out, float scaleA2, const float *scaleB2, int m,
+                              int n, int k, bsq_stream_t stream) {
+    if (m < 0 || n < 0 || k <= 0 || k % 16 || !std::isfinite(scaleA2)) return BSQ_ERR_INVALID_ARG;
+    if (m > 0 && n > 0 && !scaleB2) return BSQ_ERR_INVALID_ARG;
+    if (scaleB2 && !al4(scaleB2)) return BSQ_ERR_MISALIGNED;
+    return w4a4_common(a_packed, a_scale, w_packed, w_scale, out, scaleA2, scaleB2, m, n, k, stream);
 }
 
 bsq_status fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *row_scale, uint16_t *out, int m,

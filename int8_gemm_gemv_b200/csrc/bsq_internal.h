@@ -23,8 +23,10 @@ uint32_t take_timeouts_gemv();
 int sm_count();
 
 // ---- launchers (quant.cu) ----
-cudaError_t launch_quant_nvfp4(const uint16_t *in, uint8_t *packed, uint8_t *scale, float scale2, int m, int k,
-                               cudaStream_t s);
+// amax_dev: NULL (scale2 given), or the tensor's device amax, from which the
+// kernel derives scale2 (and writes it to scale2_out if that is not NULL)
+cudaError_t launch_quant_nvfp4(const uint16_t *in, uint8_t *packed, uint8_t *scale, float scale2,
+                               const float *amax_dev, float *scale2_out, int m, int k, cudaStream_t s);
 cudaError_t launch_quant_rowwise_fp8(const uint16_t *in, uint8_t *q, float *scale, int rows, int k,
                                      cudaStream_t s);
 cudaError_t launch_quant_blockfp8(const uint16_t *in, uint8_t *q, float *scale, int n, int k, cudaStream_t s);
@@ -43,13 +45,14 @@ cudaError_t launch_fp8_gemv_blockscaled(const uint16_t *in, const uint8_t *w, co
                                         uint16_t *out, int m, int n, int k, cudaStream_t s);
 
 // ---- launchers (gemm_*.cu) ----
+// scale_b_dev: NULL, or a device float that multiplies scale_ab in the kernel
 cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
-                             const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k,
-                             cudaStream_t s);
+                             const uint8_t *w_scale, uint16_t *out, float scale_ab, const float *scale_b_dev,
+                             int m, int n, int k, cudaStream_t s);
 // M <= 128: swapped operands, one CTA per 128 weight rows (gemm_w4a4_small.cu)
 cudaError_t launch_w4a4_gemm_small(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
-                                   const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k,
-                                   cudaStream_t s);
+                                   const uint8_t *w_scale, uint16_t *out, float scale_ab, const float *scale_b_dev,
+                                   int m, int n, int k, cudaStream_t s);
 cudaError_t launch_fp8_gemm_rowscale(const uint8_t *a, const float *a_scale, const uint8_t *w,
                                      const float *w_scale, uint16_t *out, int m, int n, int k, cudaStream_t s);
 cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const float *a_scale,

@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_w4a4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                 const __grid_constant__ CUtensorMap tmOut, int use_tma_store, uint16_t *__restrict__ out,
-                float scale_ab, int M, int N, int K) {
+                float scale_ab, const float *__restrict__ scale_b_dev, int M, int N, int K) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *out_stage = base + (size_t)STAGES * STAGE_BYTES;
@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // with TMA stores (coalesced, asynchronous).
         const int q = warp & 3, h = (warp - 4) >> 2;
         uint8_t *stage = out_stage + (warp - 4) * OUT_WARP_BYTES;
+        bool scale_read = scale_b_dev == nullptr;
         uint32_t tc = 0;
         const uint32_t tempty_leader = leader(&S->tempty);
         if (lane == 0) prefetch_tensormap(&tmOut);
@@ -280,6 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            if (!scale_read) {  // the weight scale2 from device memory, after the producer's dependency wait
+                scale_ab = __fmul_rn(scale_ab, __ldg(scale_b_dev));
+                scale_read = true;
+            }
             const uint32_t tbase = tmem + ACC_COL + ((uint32_t)(32 * q) << 16) + h * 128;
             uint32_t pk[64];  // 128 columns of this lane's row as BF16 pairs
 #pragma unroll
@@ -374,8 +379,8 @@ static int w4a4_max_pairs(cudaLaunchConfig_t cfg) {
 }
 
 cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
-                             const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k,
-                             cudaStream_t s) {
+                             const uint8_t *w_scale, uint16_t *out, float scale_ab, const float *scale_b_dev,
+                             int m, int n, int k, cudaStream_t s) {
     alignas(64) CUtensorMap tA, tB, tSA, tSB;
     const uint64_t kb = (uint64_t)k / 2, ks = (uint64_t)k / 16;
     // TMA stores need 16-byte output rows (n % 8 == 0); otherwise plain stores
@@ -417,7 +422,8 @@ cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, co
     cfg.numAttrs = 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
     cfg.gridDim = dim3(2 * pairs);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_w4a4_gemm, tA, tB, tSA, tSB, tO, use_tma_store, out, scale_ab, m, n, k);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_w4a4_gemm, tA, tB, tSA, tSB, tO, use_tma_store, out, scale_ab,
+                                       scale_b_dev, m, n, k);
     note_launch();
     return e;
 }

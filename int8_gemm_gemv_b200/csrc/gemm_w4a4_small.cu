@@ -91,7 +91,8 @@ template <int NA>
 __global__ void __launch_bounds__(kThreads, 1)
     k_w4a4_small(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFW,
-                 uint16_t *__restrict__ out, float scale_ab, int M, int N, int K) {
+                 uint16_t *__restrict__ out, float scale_ab, const float *__restrict__ scale_b_dev, int M, int N,
+                 int K) {
     using C = Cfg<NA>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -257,6 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            // the weight scale2 from device memory, after the producer's dependency wait
+            if (scale_b_dev != nullptr && tc == 0) scale_ab = __fmul_rn(scale_ab, __ldg(scale_b_dev));
             uint32_t r[HALF];
             ld_cols<HALF>(tmem + ((uint32_t)(32 * q) << 16) + h * HALF, r);
             tmem_ld_wait();
@@ -287,7 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int NA>
 cudaError_t launch_na(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
-                      const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k, cudaStream_t s) {
+                      const uint8_t *w_scale, uint16_t *out, float scale_ab, const float *scale_b_dev, int m, int n,
+                      int k, cudaStream_t s) {
     alignas(64) CUtensorMap tA, tW, tSA, tSW;
     const uint64_t kb = (uint64_t)k / 2, ks = (uint64_t)k / 16;
     // activation boxes have NA rows; rows past M are zero-filled
@@ -316,7 +320,7 @@ cudaError_t launch_na(const uint8_t *a_packed, const uint8_t *a_scale, const uin
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_w4a4_small<NA>, tA, tW, tSA, tSW, out, scale_ab, m, n, k);
+    return cudaLaunchKernelEx(&cfg, k_w4a4_small<NA>, tA, tW, tSA, tSW, out, scale_ab, scale_b_dev, m, n, k);
 }
 
 }  // namespace
@@ -329,15 +333,15 @@ uint32_t take_timeouts_gemm_w4a4_small() {
 }
 
 cudaError_t launch_w4a4_gemm_small(const uint8_t *a_packed, const uint8_t *a_scale, const uint8_t *w_packed,
-                                   const uint8_t *w_scale, uint16_t *out, float scale_ab, int m, int n, int k,
-                                   cudaStream_t s) {
+                                   const uint8_t *w_scale, uint16_t *out, float scale_ab, const float *scale_b_dev,
+                                   int m, int n, int k, cudaStream_t s) {
     cudaError_t e;
     if (m <= 32)
-        e = launch_na<32>(a_packed, a_scale, w_packed, w_scale, out, scale_ab, m, n, k, s);
+        e = launch_na<32>(a_packed, a_scale, w_packed, w_scale, out, scale_ab, scale_b_dev, m, n, k, s);
     else if (m <= 64)
-        e = launch_na<64>(a_packed, a_scale, w_packed, w_scale, out, scale_ab, m, n, k, s);
+        e = launch_na<64>(a_packed, a_scale, w_packed, w_scale, out, scale_ab, scale_b_dev, m, n, k, s);
     else
-        e = launch_na<128>(a_packed, a_scale, w_packed, w_scale, out, scale_ab, m, n, k, s);
+        e = launch_na<128>(a_packed, a_scale, w_packed, w_scale, out, scale_ab, scale_b_dev, m, n, k, s);
     note_launch();
     return e;
 }

@@ -223,17 +223,27 @@ __device__ __forceinline__ uint32_t nvfp4_codes_8(const uint4 &v, float d, const
 // registers, eight code bytes and one scale byte stored.
 __global__ void __launch_bounds__(256) k_quant_nvfp4(const uint4 *__restrict__ in, uint2 *__restrict__ packed,
                                                      uint8_t *__restrict__ sf, float scale2, float t6,
-                                                     int64_t nblocks) {
+                                                     const float *__restrict__ amax_dev,
+                                                     float *__restrict__ scale2_out, int64_t nblocks) {
     // a GEMM launched after this kernel with programmatic stream
     // serialization may start its prologue now; it reads these outputs only
     // after griddepcontrol.wait, i.e. after this grid has completed
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (amax_dev != nullptr) {
+        // the weight's scale2 from its device amax, the same FP32 steps as
+        // on the host: scale2 = amax / (6 * 448), t6 = 6 * scale2
+        scale2 = __fdiv_rn(__ldg(amax_dev), 2688.0f);
+        t6 = __fmul_rn(6.0f, scale2);
+        if (scale2_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *scale2_out = scale2;
+    }
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const Bracket t6b = bracket_of(t6);
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
         const uint4 v0 = ld_nc_v4(in + 2 * b), v1 = ld_nc_v4(in + 2 * b + 1);
         const uint32_t mx = max(amax_bits_8(v0), amax_bits_8(v1));
-        const uint8_t sc = e4m3_of_quotient(__uint_as_float(mx << 16), t6, t6b);
+        // an all-zero block has scale code 0 (also when scale2 is 0: an
+        // all-zero tensor's device amax)
+        const uint8_t sc = mx == 0 ? (uint8_t)0 : e4m3_of_quotient(__uint_as_float(mx << 16), t6, t6b);
         const float sfv = e4m3_to_f32(sc);
         uint2 codes = make_uint2(0u, 0u);
         if (sfv != 0.0f) {
@@ -596,13 +606,13 @@ int grid_for(int64_t work, int threads) {
 
 }  // namespace
 
-cudaError_t launch_quant_nvfp4(const uint16_t *in, uint8_t *packed, uint8_t *scale, float scale2, int m, int k,
-                               cudaStream_t s) {
+cudaError_t launch_quant_nvfp4(const uint16_t *in, uint8_t *packed, uint8_t *scale, float scale2,
+                               const float *amax_dev, float *scale2_out, int m, int k, cudaStream_t s) {
     const int64_t nblocks = (int64_t)m * k / 16;
     const float t6 = 6.0f * scale2;
     k_quant_nvfp4<<<grid_for(nblocks, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(in),
                                                          reinterpret_cast<uint2 *>(packed), scale, scale2, t6,
-                                                         nblocks);
+                                                         amax_dev, scale2_out, nblocks);
     note_launch();
     return cudaGetLastError();
 }

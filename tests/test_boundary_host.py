@@ -64,6 +64,14 @@ def test_validation_launches_nothing():
         (1, "quantize_bf16_to_nvfp4", (A16, A16b, A16c, 1.0, -1, 32, 0)),       # m < 0
         (2, "quantize_bf16_to_nvfp4", (ODD, A16b, A16c, 1.0, 4, 32, 0)),        # misaligned
         (0, "quantize_bf16_to_nvfp4", (None, None, None, 1.0, 0, 32, 0)),       # empty
+        (1, "quantize_bf16_to_nvfp4_devscale", (A16, A16b, A16c, None, None, 4, 32, 0)),   # amax NULL
+        (1, "quantize_bf16_to_nvfp4_devscale", (A16, A16b, A16c, A16d, None, 4, 24, 0)),   # k % 16
+        (2, "quantize_bf16_to_nvfp4_devscale", (A16, A16b, A16c, ODD, None, 4, 32, 0)),    # amax odd
+        (0, "quantize_bf16_to_nvfp4_devscale", (None, None, None, None, None, 0, 32, 0)),  # empty
+        (1, "w4a4_gemm_devscale", (A16, A16b, A16c, A16d, A16e, 1.0, None, 16, 16, 256, 0)),
+        (2, "w4a4_gemm_devscale", (A16, A16b, A16c, A16d, A16e, 1.0, ODD, 16, 16, 256, 0)),
+        (3, "w4a4_gemm_devscale", (A16, A16b, A16c, A16d, A16e, 1.0, A16, 16, 16, 272, 0)),
+        (0, "w4a4_gemm_devscale", (A16, A16b, A16c, A16d, A16e, 1.0, None, 0, 16, 256, 0)),
         (1, "w4a4_gemm", (A16, A16b, A16c, A16d, A16e, 1.0, 1.0, 16, 16, 40, 0)),
         (3, "w4a4_gemm", (A16, A16b, A16c, A16d, A16e, 1.0, 1.0, 16, 16, 272, 0)),  # k % 256
         (2, "w4a4_gemm", (A16, A16b, A16c, A16d, ODD, 1.0, 1.0, 16, 16, 256, 0)),

@@ -84,6 +84,47 @@ def test_w4a4_small_m_shapes(mnk):
     check_tol(g, ob, ab, f"w4a4 small {mnk}")
 
 
+@pytest.mark.parametrize("m", [16, 300])
+def test_w4a4_device_scale2_chain(m):
+    """Weight scale2 formed on the device (amax -> scale2 -> codes) and read
+    by the GEMM from device memory: codes, scales and scale2 equal the host
+    form; the GEMM output equals the host-scale call bit for bit."""
+    n, k = 768, 1024
+    a_bf, w_bf = synth.w4a4_inputs(m, n, k, seed=7, heavy_tailed=True)
+    wd = to_dev(w_bf)
+    amax = empty((1,), torch.float32)
+    bsq.bsq_amax_bf16(wd, w_bf.size, amax)
+    wp, wsf = empty((n, k // 2), torch.uint8), empty((n, k // 16), torch.uint8)
+    s2 = empty((1,), torch.float32)
+    bsq.quantize_bf16_to_nvfp4_devscale(wd, wp, wsf, amax, s2, n, k)
+    torch.cuda.synchronize()
+    s2_host = float(np.float32(oracle.amax_bf16(w_bf)) / np.float32(6 * 448))
+    assert float(s2.item()) == s2_host
+    owp, owsf = oracle.quant_nvfp4(w_bf, s2_host)
+    assert np.array_equal(host(wp), owp) and np.array_equal(host(wsf), owsf)
+    ap, asf = oracle.quant_nvfp4(a_bf, 1.0)
+    out_dev = bf16_out((m, n))
+    bsq.w4a4_gemm_devscale(to_dev(ap), to_dev(asf), wp, wsf, out_dev, 1.0, s2, m, n, k)
+    out_host = bf16_out((m, n))
+    bsq.w4a4_gemm(to_dev(ap), to_dev(asf), wp, wsf, out_host, 1.0, s2_host, m, n, k)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(out_dev, np.uint16), host(out_host, np.uint16))
+    ob, _, ab = oracle.w4a4_gemm(ap, asf, owp, owsf, 1.0, s2_host)
+    check_tol(host(out_dev, np.uint16), ob, ab, f"w4a4 devscale m={m}")
+
+
+def test_nvfp4_device_scale2_all_zero():
+    x = np.zeros((4, 64), np.uint16)
+    amax = empty((1,), torch.float32)
+    xd = to_dev(x)
+    bsq.bsq_amax_bf16(xd, x.size, amax)
+    p, sf = empty((4, 32), torch.uint8), empty((4, 4), torch.uint8)
+    s2 = empty((1,), torch.float32)
+    bsq.quantize_bf16_to_nvfp4_devscale(xd, p, sf, amax, s2, 4, 64)
+    torch.cuda.synchronize()
+    assert float(s2.item()) == 0.0 and not host(p).any() and not host(sf).any()
+
+
 def test_w4a4_structured_one_hot():
     """One-hot activation rows pick single weight elements: checks nibble
     order, scale placement per row and per 16-block, and the M/N tiling."""
