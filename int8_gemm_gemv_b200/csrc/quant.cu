@@ -541,29 +541,51 @@ __device__ __forceinline__ float quad_max(float a) {
     return fmaxf(a, __shfl_xor_sync(mask, a, 2));
 }
 
-__global__ void __launch_bounds__(256) k_requant_w_nvfp4_int8(const uint32_t *__restrict__ packed,
+// NVFP4 -> int8 requant: two threads per 32-block, one 16-element NVFP4
+// block each.  A block's values take only eight magnitudes,
+// v(e) = RN(RN(e2m1(e) * sf) * scale2), and the int8 code map is odd
+// (RN, rint and the clamp are symmetric).  So each thread codes the eight
+// magnitudes once and looks its sixteen codes up by nibble with byte
+// permutes: magnitude bits select from the table, the sign bit selects the
+// negated table.  The block amax is v at the largest magnitude present.
+__global__ void __launch_bounds__(256) k_requant_w_nvfp4_int8(const uint2 *__restrict__ packed,
                                                               const uint8_t *__restrict__ sf, float scale2,
-                                                              uint2 *__restrict__ q, float *__restrict__ scale,
-                                                              int64_t ngroups) {
+                                                              uint4 *__restrict__ q, float *__restrict__ scale,
+                                                              int64_t nblocks16) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t h = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; h < ngroups; h += stride) {
-        // group h: elements [8h, 8h+8) of the flattened [n, k] weight; its
-        // NVFP4 scale is that of the 16-element block h / 2
-        const uint32_t p = __ldg(packed + h);
-        const float sfv = e4m3_to_f32(__ldg(sf + (h >> 1)));
+    for (int64_t h = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; h < nblocks16; h += stride) {
+        const uint2 p = __ldg(packed + h);
+        const float sfv = e4m3_to_f32(__ldg(sf + h));
+        // largest magnitude code present (per-byte maxima of both nibbles)
+        const uint32_t mags = __vmaxu4(__vmaxu4(p.x & 0x07070707u, (p.x >> 4) & 0x07070707u),
+                                       __vmaxu4(p.y & 0x07070707u, (p.y >> 4) & 0x07070707u));
+        const uint32_t mmax = max(max(mags & 0xFFu, (mags >> 8) & 0xFFu), max((mags >> 16) & 0xFFu, mags >> 24));
+        // v(e) for e = 0..7, as four pairs
         float v[8];
-        float amax = 0.0f;
 #pragma unroll
         for (int j = 0; j < 4; j++) {
-            const float2 e = e2m1x2_to_f32x2((p >> (8 * j)) & 0xFFu);
+            const float2 e = e2m1x2_to_f32x2((uint32_t)((2 * j + 1) << 4 | (2 * j)));
             v[2 * j] = __fmul_rn(__fmul_rn(e.x, sfv), scale2);
             v[2 * j + 1] = __fmul_rn(__fmul_rn(e.y, sfv), scale2);
-            amax = fmaxf(amax, fmaxf(fabsf(v[2 * j]), fabsf(v[2 * j + 1])));
         }
-        amax = quad_max(amax);
+        const float vmax = mmax == 0 ? 0.0f : mmax == 1 ? v[1] : mmax == 2 ? v[2] : mmax == 3 ? v[3]
+                         : mmax == 4 ? v[4] : mmax == 5 ? v[5] : mmax == 6 ? v[6] : v[7];
+        const float amax = fmaxf(fabsf(vmax), __shfl_xor_sync(__activemask(), fabsf(vmax), 1));
         const float s = __fdiv_rn(amax, 127.0f);
-        q[h] = int8_codes_8(v, s, bracket_of(s));
-        if ((h & 3) == 0) scale[h >> 2] = s;
+        // table of the eight magnitudes' codes (bytes 0..7) and its negation
+        const uint2 t = int8_codes_8(v, s, bracket_of(s));
+        const uint2 tn = make_uint2(__vsub4(0u, t.x), __vsub4(0u, t.y));
+        uint32_t w[4];
+#pragma unroll
+        for (int g = 0; g < 4; g++) {
+            const uint32_t n = ((g < 2 ? p.x : p.y) >> (16 * (g & 1))) & 0xFFFFu;  // elements 4g..4g+3
+            const uint32_t sel = n & 0x7777u;
+            const uint32_t pos = __byte_perm(t.x, t.y, sel), neg = __byte_perm(tn.x, tn.y, sel);
+            const uint32_t neg_mask = __byte_perm(0x0000FF00u, 0u, (n >> 3) & 0x1111u);
+            w[g] = (pos & ~neg_mask) | (neg & neg_mask);
+        }
+        q[h] = make_uint4(w[0], w[1], w[2], w[3]);
+        if ((h & 1) == 0) scale[h >> 1] = s;
     }
 }
 
@@ -639,9 +661,9 @@ cudaError_t launch_requant_blockfp8_to_rowwise(const uint8_t *w, const float *bs
 
 cudaError_t launch_requant_w_nvfp4_int8(const uint8_t *packed, const uint8_t *sf, float scale2, int8_t *q,
                                         float *scale, int n, int k, cudaStream_t s) {
-    const int64_t ng = (int64_t)n * k / 8;
-    k_requant_w_nvfp4_int8<<<grid_for(ng, 256), 256, 0, s>>>(reinterpret_cast<const uint32_t *>(packed), sf, scale2,
-                                                             reinterpret_cast<uint2 *>(q), scale, ng);
+    const int64_t nb = (int64_t)n * k / 16;
+    k_requant_w_nvfp4_int8<<<grid_for(nb, 256), 256, 0, s>>>(reinterpret_cast<const uint2 *>(packed), sf, scale2,
+                                                             reinterpret_cast<uint4 *>(q), scale, nb);
     note_launch();
     return cudaGetLastError();
 }
