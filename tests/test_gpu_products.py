@@ -154,7 +154,7 @@ def test_w4a4_realistic_mid():
     check_tol(g[rows], ob, ab, "w4a4 512x2048x5120")
 
 
-@pytest.mark.parametrize("m", [4096, 512])
+@pytest.mark.parametrize("m", [4096, 512, 16384])
 def test_w4a4_full_size(m):
     n, k = 17408, 5120
     args = nvfp4_random(m, n, k, seed=2)

@@ -59,6 +59,16 @@ def test_quant_nvfp4_bitexact(case):
     assert np.array_equal(gp, op), f"codes differ at {np.argwhere(gp != op)[:4]}"
 
 
+def test_quant_nvfp4_largest_activation_shape_sampled_rows():
+    """16384 x 5120 activations (the largest W4A4 configuration): every
+    sampled row bit-exact."""
+    x = synth.student_t_bf16((16384, 5120), 4.0, 0, 11, outlier_frac=0.01)
+    gp, gs = gpu_nvfp4(x, 1.0)
+    rows = np.array([0, 1, 4095, 4096, 8191, 12345, 16383])
+    op, os_ = oracle.quant_nvfp4(x[rows], 1.0)
+    assert np.array_equal(gs[rows], os_) and np.array_equal(gp[rows], op)
+
+
 def test_quant_nvfp4_weight_scale2_from_device_amax():
     x = synth.normal_bf16((512, 1024), 0.02, 3, 2)
     amax = empty((1,), torch.float32)
