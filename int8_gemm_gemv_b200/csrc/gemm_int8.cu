@@ -5,18 +5,26 @@
 // The scales change every 32 K, which is exactly one int8 MMA K step, so the
 // tensor cores cannot accumulate across blocks.  Each 128x128x32 MMA writes a
 // fresh int32 partial into one of four tensor-memory buffers (4 x 128
-// columns); eight "fold" warps read each partial back and fold it into FP32
+// columns); sixteen "fold" warps read each partial back and fold it into FP32
 // registers with its two scales while the tensor cores already compute the
-// next ones.  The fold (one convert, one multiply, one FMA per output and
-// block) on the CUDA cores is the bound of this kernel, not the int8 MMA.
+// next ones.  The fold (one convert, one scale product, one FMA per output
+// and block) on the CUDA cores is the bound of this kernel, not the int8 MMA.
 //
 //   warp 0       TMA producer: A, W tiles (128 x 128 B) and their scale tiles
 //                (128 rows x 4 FP32) into a 6-stage ring
 //   warp 1       MMA issuer
-//   warp 2       rewrites each stage's W-scale tile from [n][4] to [4][n] so
-//                the fold warps read 4 columns per shared-memory load
-//   warps 4..11  fold + epilogue; warp w owns tensor-memory lane quarter
-//                w % 4 (rows) and column half (w - 4) / 4
+//   warp 2       rewrites each stage's W-scale tile from [n][4] to [4][n]
+//   warps 4..19  fold + epilogue; warp w owns tensor-memory lane quarter
+//                w % 4 (rows) and column quarter (w - 4) / 4: a 32 x 32
+//                sub-tile of every partial
+//
+// The fold reads partials with the 16-lane x 256-bit tensor-memory shape: a
+// thread holds 4 rows x 8 columns of its warp's sub-tile, so it needs 4 row
+// scales and 4 column-scale pairs per block (each pair shared by 8 lanes).
+// The two 16-row halves of a partial are loaded one ahead of the other, so
+// each half is folded while the next is in flight.  Four fold warps per
+// SM sub-partition hide the remaining latency; to fit them, warps 0-3 give
+// up registers (setmaxnreg).
 #include "bsq_common.cuh"
 
 namespace bsq {
@@ -30,8 +38,13 @@ constexpr int SA_BYTES = BM * 16, SW_BYTES = BN * 16;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SA_BYTES + SW_BYTES;
 constexpr int NACC = 4;  // tensor-memory partial buffers of 128 columns
 constexpr int TMEM_COLS = 512;
-constexpr int NFOLD = 8;
+constexpr int NFOLD = 16;
 constexpr int kThreads = 32 * (4 + NFOLD);
+// Register split: the block is launched with kLaunchRegs per thread; warps
+// 0-3 (one warpgroup) drop to kCtlRegs and the two fold warpgroups take the
+// rest.  The launcher checks the compiled count before the first launch.
+constexpr int kLaunchRegs = 96, kCtlRegs = 48, kFoldRegs = 104;
+static_assert(128 * kCtlRegs + 32 * NFOLD * kFoldRegs <= kThreads * kLaunchRegs, "register split");
 
 static __device__ unsigned int g_timeouts;
 
@@ -48,6 +61,13 @@ struct Smem {
 constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Smem);
 
 __device__ __forceinline__ bool aborted(volatile Smem *s) { return s->abort != 0; }
+
+template <int R> __device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <int R> __device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
 
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
     float2 d;
@@ -106,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = S->tmem_base;
+    if (warp < 4) setmaxnreg_dec<kCtlRegs>();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -197,86 +218,104 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= 4) {
         // ------------------------------------------------ fold + epilogue
+        setmaxnreg_inc<kFoldRegs>();
         const int q = warp & 3, h = (warp - 4) >> 2;
-        const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+        // this warp's 32 x 32 sub-tile: lanes 32q.., columns 32h..
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + 32 * h;
+        const int r0 = 32 * q + (lane >> 2);  // rows r0, r0 + 8 (upper half), r0 + 16, r0 + 24 (lower half)
+        const int c0 = 32 * h + 2 * (lane & 3);  // columns c0 + 8g, c0 + 8g + 1
         uint32_t it = 0, gs = 0;
         bool ok = true;
+        uint32_t RA[16], RB[16];  // upper / lower 16 rows of the sub-tile
+        float2 acc[16];           // [row 0..3][group 0..3], a column pair each
+        auto wait_full = [&](uint32_t g) -> bool {
+            if (!mbar_wait(&S->acc_full[g % NACC], (g / NACC) & 1, &g_timeouts) || aborted(S)) return false;
+            tc_fence_after();
+            return true;
+        };
+        // rows u0, u0 + 1 of the accumulator from one 16-row half
+        auto fold_half = [&](const uint32_t (&R)[16], int u0, float s0, float s1, const float2 (&w2)[4]) {
+#pragma unroll
+            for (int g = 0; g < 4; g++) {
+                const float2 c0v = mul2(make_float2(s0, s0), w2[g]);
+                const float2 c1v = mul2(make_float2(s1, s1), w2[g]);
+                acc[4 * u0 + g] = fma2(make_float2((float)(int)R[4 * g], (float)(int)R[4 * g + 1]), c0v, acc[4 * u0 + g]);
+                acc[4 * u0 + 4 + g] =
+                    fma2(make_float2((float)(int)R[4 * g + 2], (float)(int)R[4 * g + 3]), c1v, acc[4 * u0 + 4 + g]);
+            }
+        };
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             const int mt = t % tiles_m, nt = t / tiles_m;
-            float2 acc[32];
 #pragma unroll
-            for (int i = 0; i < 32; i++) acc[i] = make_float2(0.0f, 0.0f);
+            for (int i = 0; i < 16; i++) acc[i] = make_float2(0.0f, 0.0f);
+            if (!wait_full(gs)) {
+                ok = false;
+                break;
+            }
+            tmem_ld_16x256b_x4(tq + (gs % NACC) * BN, RA);
+            tmem_ld_wait();
             for (int kb = 0; kb < nkb && ok; kb++, it++) {
                 const int s = it % STAGES;
                 if (!mbar_wait(&S->swready[s], (it / STAGES) & 1, &g_timeouts) || aborted(S)) {
                     ok = false;
                     break;
                 }
-                const float4 sa4 = reinterpret_cast<const float4 *>(sa_tile(s))[32 * q + lane];
-                const float *sw = sw_tile(s) + 64 * h;
-#pragma unroll 1
+                const float *sat = sa_tile(s);
+                const bool last = kb == nkb - 1;
+#pragma unroll
                 for (int j = 0; j < 4; j++, gs++) {
-                    const int b = gs % NACC;
-                    if (!mbar_wait(&S->acc_full[b], (gs / NACC) & 1, &g_timeouts) || aborted(S)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    uint32_t r0[32], r1[32];
-                    tmem_ld_32x32b_x32(tmem + b * BN + lane_off + 64 * h, r0);
-                    tmem_ld_32x32b_x32(tmem + b * BN + lane_off + 64 * h + 32, r1);
+                    // Upper half of block gs is in RA.  Load the lower half,
+                    // fold the upper; then load the upper half of the next
+                    // block while the lower one is folded.
+                    const uint32_t b = gs % NACC;
+                    tmem_ld_16x256b_x4(tq + (16u << 16) + b * BN, RB);
+                    float sr[4];
+#pragma unroll
+                    for (int u = 0; u < 4; u++) sr[u] = sat[(r0 + 8 * u) * 4 + j];
+                    float2 w2[4];
+                    const float *swt = sw_tile(s) + j * BN + c0;
+#pragma unroll
+                    for (int g = 0; g < 4; g++) w2[g] = *reinterpret_cast<const float2 *>(swt + 8 * g);
+                    fold_half(RA, 0, sr[0], sr[1], w2);
                     tmem_ld_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S->acc_empty[b]);
-                    const float saj = j == 0 ? sa4.x : j == 1 ? sa4.y : j == 2 ? sa4.z : sa4.w;
-                    const float2 sa2 = make_float2(saj, saj);
-                    const float4 *swj = reinterpret_cast<const float4 *>(sw + j * BN);
-#pragma unroll
-                    for (int i = 0; i < 8; i++) {
-                        const float4 w4 = swj[i];
-                        const float2 s01 = mul2(sa2, make_float2(w4.x, w4.y));
-                        const float2 s23 = mul2(sa2, make_float2(w4.z, w4.w));
-                        acc[2 * i] = fma2(make_float2((float)(int)r0[4 * i], (float)(int)r0[4 * i + 1]), s01, acc[2 * i]);
-                        acc[2 * i + 1] =
-                            fma2(make_float2((float)(int)r0[4 * i + 2], (float)(int)r0[4 * i + 3]), s23, acc[2 * i + 1]);
+                    const bool nxt = !(last && j == 3);
+                    if (nxt) {
+                        if (!wait_full(gs + 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tmem_ld_16x256b_x4(tq + ((gs + 1) % NACC) * BN, RA);
                     }
-#pragma unroll
-                    for (int i = 0; i < 8; i++) {
-                        const float4 w4 = swj[8 + i];
-                        const float2 s01 = mul2(sa2, make_float2(w4.x, w4.y));
-                        const float2 s23 = mul2(sa2, make_float2(w4.z, w4.w));
-                        acc[16 + 2 * i] =
-                            fma2(make_float2((float)(int)r1[4 * i], (float)(int)r1[4 * i + 1]), s01, acc[16 + 2 * i]);
-                        acc[16 + 2 * i + 1] = fma2(make_float2((float)(int)r1[4 * i + 2], (float)(int)r1[4 * i + 3]),
-                                                   s23, acc[16 + 2 * i + 1]);
-                    }
+                    fold_half(RB, 2, sr[2], sr[3], w2);
+                    if (nxt) tmem_ld_wait();
                 }
+                if (!ok) break;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S->empty[s]);
             }
             if (!ok) {
+                tmem_ld_wait();
                 if (lane == 0) S->abort = 1;
                 break;
             }
-            const int row = mt * BM + 32 * q + lane;
-            const int n0 = nt * BN + 64 * h;
-            if (row < M) {
+            // epilogue: rows r0 + 8u, column pairs c0 + 8g
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int row = mt * BM + r0 + 8 * u;
+                if (row >= M) continue;
                 uint16_t *orow = out + (int64_t)row * N;
-                if ((N % 8) == 0 && n0 + 64 <= N) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + n0);
 #pragma unroll
-                    for (int i = 0; i < 8; i++)
-                        dst[i] = make_uint4(pack_bf16x2(acc[4 * i].x, acc[4 * i].y),
-                                            pack_bf16x2(acc[4 * i + 1].x, acc[4 * i + 1].y),
-                                            pack_bf16x2(acc[4 * i + 2].x, acc[4 * i + 2].y),
-                                            pack_bf16x2(acc[4 * i + 3].x, acc[4 * i + 3].y));
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; i++) {
-                        if (n0 + 2 * i < N) orow[n0 + 2 * i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[i].x));
-                        if (n0 + 2 * i + 1 < N)
-                            orow[n0 + 2 * i + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[i].y));
+                for (int g = 0; g < 4; g++) {
+                    const int col = nt * BN + c0 + 8 * g;
+                    const float2 v = acc[4 * u + g];
+                    if ((N & 1) == 0 && col + 1 < N) {
+                        *reinterpret_cast<uint32_t *>(orow + col) = pack_bf16x2(v.x, v.y);
+                    } else {
+                        if (col < N) orow[col] = __bfloat16_as_ushort(__float2bfloat16_rn(v.x));
+                        if (col + 1 < N) orow[col + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(v.y));
                     }
                 }
             }
@@ -314,7 +353,13 @@ cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_int8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        // The register split is only valid for a block launched with exactly
+        // kLaunchRegs registers per thread.
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, k_int8_gemm);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(k_int8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }

@@ -531,16 +531,6 @@ __device__ __forceinline__ uint2 int8_codes_8(const float (&v)[8], float s, cons
     return make_uint2(w0, w1);
 }
 
-// Both int8 kernels give four threads to each 32-element block, eight
-// elements per thread; the block amax is a two-step shuffle inside the
-// quad, and one thread of the quad stores the block scale.  The grid stride
-// is a multiple of four, so a quad stays together to the last iteration.
-__device__ __forceinline__ float quad_max(float a) {
-    const unsigned mask = __activemask();
-    a = fmaxf(a, __shfl_xor_sync(mask, a, 1));
-    return fmaxf(a, __shfl_xor_sync(mask, a, 2));
-}
-
 // NVFP4 -> int8 requant: two threads per 32-block, one 16-element NVFP4
 // block each.  A block's values take only eight magnitudes,
 // v(e) = RN(RN(e2m1(e) * sf) * scale2), and the int8 code map is odd
@@ -589,6 +579,11 @@ __global__ void __launch_bounds__(256) k_requant_w_nvfp4_int8(const uint2 *__res
     }
 }
 
+// Activations -> int8: four threads to each 32-element block, eight
+// elements per thread; the block amax is a two-step shuffle of magnitude
+// bits inside the quad, and the quad's first thread stores the block scale.
+// The grid stride is a multiple of four, so a quad stays together to the
+// last iteration.
 __global__ void __launch_bounds__(256) k_quant_act_int8_per32(const uint16_t *__restrict__ a, uint2 *__restrict__ q,
                                                               float *__restrict__ scale, int64_t ngroups) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
