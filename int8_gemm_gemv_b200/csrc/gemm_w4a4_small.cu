@@ -58,6 +58,12 @@ struct Cfg {
     static_assert(NA <= SF_COL, "accumulator columns");
 };
 
+// Rows of the activation boxes: NA, or 1 for a one-row activation.
+template <int NA>
+__host__ __device__ constexpr int act_box_rows(int m) {
+    return m == 1 ? 1 : NA;
+}
+
 struct Smem {
     uint64_t full[8], sfready[8], empty[8];
     uint64_t tfull, tempty, drain;
@@ -106,6 +112,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_tiles = (N + BW - 1) / BW;
     const int nkb = K / 256;
+    // Activation boxes have NA rows, the rows past M zero-filled by the
+    // copy -- except for a single row (M = 1), where a one-row box is much
+    // faster: its padding rows are zeroed here once and never copied.
+    const int ma = act_box_rows<NA>(M);
+    if (ma < NA) {
+        for (int s = 0; s < STAGES; s++) {
+            for (int i = ma * (BK_BYTES / 16) + threadIdx.x; i < NA * (BK_BYTES / 16); i += kThreads)
+                reinterpret_cast<uint4 *>(a_tile(s))[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = ma + threadIdx.x; i < NA; i += kThreads)
+                reinterpret_cast<uint4 *>(sfa_tile(s))[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+    }
+    const uint32_t data_bytes = W_BYTES + SFW_BYTES + (uint32_t)ma * (BK_BYTES + 16);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
@@ -148,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&S->full[s], C::DATA_BYTES);
+                    mbar_arrive_expect_tx(&S->full[s], data_bytes);
                     tma_load_2d(w_tile(s), &tmW, &S->full[s], kb * BK_BYTES, t * BW);
                     tma_load_2d(a_tile(s), &tmA, &S->full[s], kb * BK_BYTES, 0);
                     tma_load_2d(sfw_tile(s), &tmSFW, &S->full[s], kb * 16, t * BW);
@@ -294,10 +314,10 @@ cudaError_t launch_na(const uint8_t *a_packed, const uint8_t *a_scale, const uin
                       int k, cudaStream_t s) {
     alignas(64) CUtensorMap tA, tW, tSA, tSW;
     const uint64_t kb = (uint64_t)k / 2, ks = (uint64_t)k / 16;
-    // activation boxes have NA rows; rows past M are zero-filled
-    if (!make_tmap_2d(&tA, a_packed, 1, kb, m, kb, BK_BYTES, NA, true, false) ||
+    const uint32_t ma = (uint32_t)act_box_rows<NA>(m);
+    if (!make_tmap_2d(&tA, a_packed, 1, kb, m, kb, BK_BYTES, ma, true, false) ||
         !make_tmap_2d(&tW, w_packed, 1, kb, n, kb, BK_BYTES, BW, true, false) ||
-        !make_tmap_2d(&tSA, a_scale, 1, ks, m, ks, 16, NA, false, false) ||
+        !make_tmap_2d(&tSA, a_scale, 1, ks, m, ks, 16, ma, false, false) ||
         !make_tmap_2d(&tSW, w_scale, 1, ks, n, ks, 16, BW, false, false))
         return cudaErrorInvalidValue;
     static bool attr_done[64] = {};

@@ -22,6 +22,13 @@ namespace bsq {
 
 namespace {
 
+// Grid-stride quantisers take this many independent units per thread and
+// pass, so several loads per thread are in flight at once.
+#ifndef BSQ_QUANT_UNROLL
+#define BSQ_QUANT_UNROLL 2
+#endif
+constexpr int kQuantUnroll = BSQ_QUANT_UNROLL;
+
 __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
     uint4 r;
     asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -238,22 +245,37 @@ __global__ void __launch_bounds__(256) k_quant_nvfp4(const uint4 *__restrict__ i
     }
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const Bracket t6b = bracket_of(t6);
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
-        const uint4 v0 = ld_nc_v4(in + 2 * b), v1 = ld_nc_v4(in + 2 * b + 1);
-        const uint32_t mx = max(amax_bits_8(v0), amax_bits_8(v1));
-        // an all-zero block has scale code 0 (also when scale2 is 0: an
-        // all-zero tensor's device amax)
-        const uint8_t sc = mx == 0 ? (uint8_t)0 : e4m3_of_quotient(__uint_as_float(mx << 16), t6, t6b);
-        const float sfv = e4m3_to_f32(sc);
-        uint2 codes = make_uint2(0u, 0u);
-        if (sfv != 0.0f) {
-            const float d = __fmul_rn(sfv, scale2);
-            const Bracket br = bracket_of(d);
-            codes.x = nvfp4_codes_8(v0, d, br);
-            codes.y = nvfp4_codes_8(v1, d, br);
+    // kQuantUnroll blocks per thread and pass, all loads issued first
+    for (int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b0 < nblocks; b0 += kQuantUnroll * stride) {
+        uint4 v[kQuantUnroll][2];
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; u++) {
+            const int64_t b = b0 + u * stride;
+            v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
+            if (b < nblocks) {
+                v[u][0] = ld_nc_v4(in + 2 * b);
+                v[u][1] = ld_nc_v4(in + 2 * b + 1);
+            }
         }
-        packed[b] = codes;
-        sf[b] = sc;
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; u++) {
+            const int64_t b = b0 + u * stride;
+            if (b >= nblocks) break;
+            const uint32_t mx = max(amax_bits_8(v[u][0]), amax_bits_8(v[u][1]));
+            // an all-zero block has scale code 0 (also when scale2 is 0: an
+            // all-zero tensor's device amax)
+            const uint8_t sc = mx == 0 ? (uint8_t)0 : e4m3_of_quotient(__uint_as_float(mx << 16), t6, t6b);
+            const float sfv = e4m3_to_f32(sc);
+            uint2 codes = make_uint2(0u, 0u);
+            if (sfv != 0.0f) {
+                const float d = __fmul_rn(sfv, scale2);
+                const Bracket br = bracket_of(d);
+                codes.x = nvfp4_codes_8(v[u][0], d, br);
+                codes.y = nvfp4_codes_8(v[u][1], d, br);
+            }
+            packed[b] = codes;
+            sf[b] = sc;
+        }
     }
 }
 
@@ -587,17 +609,29 @@ __global__ void __launch_bounds__(256) k_requant_w_nvfp4_int8(const uint2 *__res
 __global__ void __launch_bounds__(256) k_quant_act_int8_per32(const uint16_t *__restrict__ a, uint2 *__restrict__ q,
                                                               float *__restrict__ scale, int64_t ngroups) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t h = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; h < ngroups; h += stride) {
-        const uint4 x = ld_nc_v4(a + h * 8);
-        float v[8];
-        unpack_bf16_8(x, v);
-        uint32_t mx = amax_bits_8(x);
-        const unsigned mask = __activemask();
-        mx = max(mx, __shfl_xor_sync(mask, mx, 1));
-        mx = max(mx, __shfl_xor_sync(mask, mx, 2));
-        const float s = __fdiv_rn(__uint_as_float(mx << 16), 127.0f);
-        q[h] = int8_codes_8(v, s, bracket_of(s));
-        if ((h & 3) == 0) scale[h >> 2] = s;
+    // kQuantUnroll groups per thread and pass, all loads issued first; a
+    // quad's four groups are in or out of range together (ngroups % 4 == 0)
+    for (int64_t h0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; h0 < ngroups; h0 += kQuantUnroll * stride) {
+        uint4 x[kQuantUnroll];
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; u++) {
+            const int64_t h = h0 + u * stride;
+            x[u] = h < ngroups ? ld_nc_v4(a + h * 8) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; u++) {
+            const int64_t h = h0 + u * stride;
+            if (h >= ngroups) break;
+            float v[8];
+            unpack_bf16_8(x[u], v);
+            uint32_t mx = amax_bits_8(x[u]);
+            const unsigned mask = __activemask();
+            mx = max(mx, __shfl_xor_sync(mask, mx, 1));
+            mx = max(mx, __shfl_xor_sync(mask, mx, 2));
+            const float s = __fdiv_rn(__uint_as_float(mx << 16), 127.0f);
+            q[h] = int8_codes_8(v, s, bracket_of(s));
+            if ((h & 3) == 0) scale[h >> 2] = s;
+        }
     }
 }
 
@@ -627,7 +661,7 @@ cudaError_t launch_quant_nvfp4(const uint16_t *in, uint8_t *packed, uint8_t *sca
                                const float *amax_dev, float *scale2_out, int m, int k, cudaStream_t s) {
     const int64_t nblocks = (int64_t)m * k / 16;
     const float t6 = 6.0f * scale2;
-    k_quant_nvfp4<<<grid_for(nblocks, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(in),
+    k_quant_nvfp4<<<grid_for((nblocks + kQuantUnroll - 1) / kQuantUnroll, 256), 256, 0, s>>>(reinterpret_cast<const uint4 *>(in),
                                                          reinterpret_cast<uint2 *>(packed), scale, scale2, t6,
                                                          amax_dev, scale2_out, nblocks);
     note_launch();
@@ -666,7 +700,7 @@ cudaError_t launch_requant_w_nvfp4_int8(const uint8_t *packed, const uint8_t *sf
 cudaError_t launch_quant_act_int8_per32(const uint16_t *a, int8_t *q, float *scale, int m, int k,
                                         cudaStream_t s) {
     const int64_t ng = (int64_t)m * k / 8;
-    k_quant_act_int8_per32<<<grid_for(ng, 256), 256, 0, s>>>(a, reinterpret_cast<uint2 *>(q), scale, ng);
+    k_quant_act_int8_per32<<<grid_for((ng + kQuantUnroll - 1) / kQuantUnroll, 256), 256, 0, s>>>(a, reinterpret_cast<uint2 *>(q), scale, ng);
     note_launch();
     return cudaGetLastError();
 }
