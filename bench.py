@@ -44,6 +44,7 @@ WORKLOADS = {
 L2_BYTES = 126 * 1024 * 1024
 # dense tensor-core throughput relative to BF16 (NVIDIA B200 datasheet ratios)
 RATIO_FP4, RATIO_FP8, RATIO_INT8 = 4.0, 2.0, 2.0
+SM_MAX_MHZ = 1965  # B200 clocks.max.sm
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -544,11 +545,16 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
     out = torch.empty((m, n), dtype=torch.int16, device=dev)
     t = time_launches(torch, stream, lambda: bsq.int8_blockscaled_gemm(ai, wi, ais, wis, out, m, n, k, stream), 5)
     tops = 2.0 * m * n * k / t / 1e12
-    # fold bound: one convert + one multiply + one FMA per output and 32-block
-    # on 148 SMs x 128 FP32 lanes at the measured clock
+    # The fold's own roofline: two FP32 lane operations (the scale product and
+    # the FMA) per output and 32-block, against every SM's 128 FP32 lanes at
+    # the maximum SM clock; the int32 -> FP32 conversions run on the ALU pipe.
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    fold_peak = sms * 128 * SM_MAX_MHZ * 1e6
+    fold_rate = 2.0 * m * n * (k // 32) / t
     rows[f"a7_int8_blockscaled_gemm_{m}x{n}x{k}"] = {
         "us": round(t * 1e6, 1), "tops": round(tops, 1), "frac_int8": round(tops / (bf16 * RATIO_INT8), 4),
-        "bound": "alu (per-32 FP32 fold on CUDA cores)"}
+        "fold_gops": round(fold_rate / 1e9, 1), "fold_peak_gops": round(fold_peak / 1e9, 1),
+        "frac_fold": round(fold_rate / fold_peak, 4), "bound": "alu (per-32 FP32 fold on CUDA cores)"}
     return rows
 
 

@@ -298,7 +298,7 @@ def run_int8(a, w, sa, sw):
     return host(out, np.uint16)
 
 
-@pytest.mark.parametrize("mnk", [(64, 128, 128), (200, 300, 640), (129, 136, 1024)])
+@pytest.mark.parametrize("mnk", [(64, 128, 128), (200, 300, 640), (129, 136, 1024), (1, 130, 256), (77, 131, 384)])
 def test_int8_small_and_ragged(mnk):
     m, n, k = mnk
     a_bf, w_bf = synth.w4a8_inputs(m, n, k, seed=1)
