@@ -239,8 +239,7 @@ uint64_t bsq_debug_launch_count(void) { return bsq::g_launches.load(std::memory_
 uint32_t bsq_debug_take_timeouts(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return 0xFFFFFFFFu;
     return bsq::take_timeouts_gemm_w4a4() | bsq::take_timeouts_gemm_w4a4_small() | bsq::take_timeouts_gemm_fp8() |
-           bsq::take_timeouts_gemm_int8() |
-           bsq::take_timeouts_gemv();
+           bsq::take_timeouts_gemm_int8() | bsq::take_timeouts_gemv() | bsq::take_timeouts_quant();
 }
 
 }  // extern "C"

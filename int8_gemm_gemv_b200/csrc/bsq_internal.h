@@ -14,6 +14,7 @@ void note_launch();
 // Per-file flags of bounded waits that ran out (read and cleared with a
 // device synchronisation; used by tests only).
 uint32_t take_timeouts_gemm_w4a4();
+uint32_t take_timeouts_quant();
 uint32_t take_timeouts_gemm_w4a4_small();
 uint32_t take_timeouts_gemm_fp8();
 uint32_t take_timeouts_gemm_int8();

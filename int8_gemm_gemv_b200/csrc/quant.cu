@@ -508,6 +508,58 @@ __global__ void __launch_bounds__(kReqThreads) k_requant_blockfp8_to_rowwise(con
             requant_codes_16(dequant_16(ld_nc_v4(wr + c * 16), __ldg(srow + (c >> 3))), s, br);
 }
 
+// Rows of up to kReqSmemMaxK codes: one CTA of kReqRowThreads per row.  One
+// bulk copy brings the whole row into shared memory, so every CTA has its
+// row in flight at once and many rows are in flight per SM; pass 1 finds the
+// amax of the BF16 transient, pass 2 writes the codes, both from shared
+// memory.
+constexpr int kReqRowThreads = 64;
+constexpr int kReqSmemMaxK = 48 * 1024;
+
+static __device__ unsigned int g_quant_timeouts;
+
+__global__ void __launch_bounds__(kReqRowThreads) k_requant_blockfp8_rows_smem(const uint8_t *__restrict__ w,
+                                                                              const float *__restrict__ bscale,
+                                                                              uint8_t *__restrict__ q,
+                                                                              float *__restrict__ scale, int k) {
+    extern __shared__ __align__(16) uint8_t srow[];
+    __shared__ uint64_t bar;
+    __shared__ uint32_t red[kReqRowThreads / 32];
+    __shared__ float ssc[kReqSmemMaxK / 128];
+    const int64_t row = blockIdx.x;
+    const int t = threadIdx.x;
+    if (t == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (t == 0) {
+        mbar_arrive_expect_tx(&bar, (uint32_t)k);
+        bulk_load_g2s(srow, w + row * k, (uint32_t)k, &bar);
+    }
+    // the row's block scales (one per 128 codes = 8 chunks), while the row is in flight
+    const int kb = k >> 7;
+    const float *srs = bscale + (row >> 7) * kb;
+    for (int i = t; i < kb; i += kReqRowThreads) ssc[i] = __ldg(srs + i);
+    __syncthreads();
+    const int nch = k >> 4;
+    // a copy that has not landed within the wait limit is reported through
+    // the timeout flag; the whole CTA leaves together
+    if (!__syncthreads_and(mbar_wait(&bar, 0, &g_quant_timeouts))) return;
+    const uint4 *sv = reinterpret_cast<const uint4 *>(srow);
+    uint32_t mx = 0;
+    for (int c = t; c < nch; c += kReqRowThreads) {
+        const Bf16x16 d = dequant_16(sv[c], ssc[c >> 3]);
+        mx = max(mx, max(amax_bits_8(d.a), amax_bits_8(d.b)));
+    }
+    mx = cta_max_once<kReqRowThreads>(mx, red);
+    const float s = __fdiv_rn(__uint_as_float(mx << 16), 448.0f);
+    if (t == 0) scale[row] = s;
+    const Bracket br = bracket_of(s);
+    uint4 *qr = reinterpret_cast<uint4 *>(q + row * k);
+    for (int c = t; c < nch; c += kReqRowThreads) qr[c] = requant_codes_16(dequant_16(sv[c], ssc[c >> 3]), s, br);
+}
+
 // ---------------------------------------------------------------------------
 // int8 per-32 blocks, one thread per block.
 
@@ -683,7 +735,10 @@ cudaError_t launch_quant_blockfp8(const uint16_t *in, uint8_t *q, float *scale, 
 
 cudaError_t launch_requant_blockfp8_to_rowwise(const uint8_t *w, const float *bscale, int n, int k, uint8_t *q,
                                                float *scale, cudaStream_t s) {
-    k_requant_blockfp8_to_rowwise<<<n, kReqThreads, 0, s>>>(w, bscale, q, scale, k);
+    if (k <= kReqSmemMaxK)
+        k_requant_blockfp8_rows_smem<<<n, kReqRowThreads, k, s>>>(w, bscale, q, scale, k);
+    else
+        k_requant_blockfp8_to_rowwise<<<n, kReqThreads, 0, s>>>(w, bscale, q, scale, k);
     note_launch();
     return cudaGetLastError();
 }
@@ -703,6 +758,13 @@ cudaError_t launch_quant_act_int8_per32(const uint16_t *a, int8_t *q, float *sca
     k_quant_act_int8_per32<<<grid_for((ng + kQuantUnroll - 1) / kQuantUnroll, 256), 256, 0, s>>>(a, reinterpret_cast<uint2 *>(q), scale, ng);
     note_launch();
     return cudaGetLastError();
+}
+
+uint32_t take_timeouts_quant() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_quant_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+    cudaMemcpyToSymbol(g_quant_timeouts, &zero, sizeof(zero));
+    return v;
 }
 
 cudaError_t launch_amax_bf16(const uint16_t *x, size_t count, float *amax, cudaStream_t s) {

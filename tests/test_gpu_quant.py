@@ -137,6 +137,23 @@ def test_requant_blockfp8_to_rowwise_bitexact_and_passthrough():
     assert np.array_equal(host(q), before)
 
 
+@pytest.mark.parametrize("nk", [(256, 128), (128, 384), (128, 49280)])
+def test_requant_blockfp8_to_rowwise_row_lengths(nk):
+    # one-block rows, an odd number of blocks, and rows longer than the
+    # shared-memory row buffer (the register path); row 3 is all zero
+    n, k = nk
+    x = synth.normal_bf16((n, k), 0.02, 0, 11)
+    x[3, :] = 0
+    w, S = oracle.quant_blockfp8(x)
+    q, s = empty(w.shape, torch.uint8), empty((n,), torch.float32)
+    bsq.requant_blockfp8_to_rowwise(bsq.BSQ_FP8_BLOCK_SCALED, to_dev(w), to_dev(S), n, k, q, s)
+    torch.cuda.synchronize()
+    oq, os_ = oracle.requant_blockfp8_to_rowwise(w, S)
+    assert np.array_equal(host(s), os_)
+    assert np.array_equal(host(q), oq)
+    assert bsq.debug_take_timeouts() == 0
+
+
 @pytest.mark.parametrize("shape", [(5120, 17408), (40, 1056)])
 def test_requant_w_nvfp4_int8_bitexact(shape):
     x = synth.normal_bf16(shape, 0.02, 0, 6)
