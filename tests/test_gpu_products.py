@@ -298,7 +298,10 @@ def run_int8(a, w, sa, sw):
     return host(out, np.uint16)
 
 
-@pytest.mark.parametrize("mnk", [(64, 128, 128), (200, 300, 640), (129, 136, 1024), (1, 130, 256), (77, 131, 384)])
+# (128, 20224, 128) has 158 tiles: more than one per SM, so some CTAs take a
+# second tile
+@pytest.mark.parametrize("mnk", [(64, 128, 128), (200, 300, 640), (129, 136, 1024), (1, 130, 256), (77, 131, 384),
+                                 (128, 20224, 128)])
 def test_int8_small_and_ragged(mnk):
     m, n, k = mnk
     a_bf, w_bf = synth.w4a8_inputs(m, n, k, seed=1)
