@@ -240,7 +240,9 @@ BSQ_API bsq_status quant_act_int8_per32(const uint16_t *a, int8_t *a_i8, float *
  *   C[i,j] = sum_b (exact int32 sum_{k in b} a*w) * a_scale[i,b] * w_scale[j,b]
  * Int8 tensor cores give the exact per-block partials; the FP32 fold runs
  * on the CUDA cores.  All pointers 16-byte aligned.
- * Errors: k % 32 != 0 -> INVALID_ARG; k % 128 != 0 -> UNSUPPORTED.
+ * Errors: k % 32 != 0 -> INVALID_ARG; k % 128 != 0 -> UNSUPPORTED.  The
+ * kernel's register split needs the build's register count; a library
+ * built with another count refuses to launch and returns BSQ_ERR_CUDA.
  * ---------------------------------------------------------------------- */
 BSQ_API bsq_status int8_blockscaled_gemm(const int8_t *a_i8, const int8_t *w_i8,
                                  const float *a_scale, const float *w_scale,
