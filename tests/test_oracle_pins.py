@@ -329,6 +329,44 @@ def test_nvfp4_zero_and_weight_scale2():
     assert torch_e4m3_decode(sf).max() >= 416
 
 
+def _torch_amax(bits: np.ndarray) -> float:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16).copy()).view(torch.bfloat16)
+    return float(t.to(torch.float32).abs().max().item()) if t.numel() else 0.0
+
+
+def test_amax_bf16_matches_torch_abs_max():
+    """The weight scale2 of gemm_fp4.rs (weight_scale_2 = amax / (6*448))
+    rests on amax = max |x| over the whole tensor.  Pinned two-sided against
+    torch's BF16 decode + abs + max: the largest magnitude negative and in
+    the last element (a missing abs or a skipped tail under-estimates it), a
+    positive maximum at index 0, BF16 subnormals only, -0 and +0 only, a
+    single element, and seeded random tensors of odd lengths."""
+    g = np.random.default_rng(11)
+    cases = []
+    x = synth.normal_bf16((1, 1001), 1.0, 3, 9).ravel().copy()
+    xf = f32(x)
+    big = np.float32(-2.0 * np.abs(xf).max())
+    x[-1] = bf16(big).reshape(-1)[0]
+    cases.append((x, abs(float(big))))
+    y = synth.normal_bf16((1, 777), 0.5, 4, 9).ravel().copy()
+    y[0] = bf16(np.float32(9.5)).reshape(-1)[0]
+    cases.append((y, 9.5))
+    sub = (g.integers(1, 0x7F, 257).astype(np.uint16) | (g.integers(0, 2, 257).astype(np.uint16) << 15))
+    cases.append((sub, None))
+    cases.append((np.array([0x8000, 0x0000, 0x8000], np.uint16), 0.0))
+    cases.append((bf16(np.float32([-3.25])).reshape(-1), 3.25))
+    for n in (15, 16, 17, 4095):
+        cases.append((synth.normal_bf16((1, n), 0.02, 5, n).ravel().copy(), None))
+    for bits, expect in cases:
+        got = oracle.amax_bf16(bits)
+        ref = _torch_amax(bits)
+        assert got == ref, (got, ref)
+        if expect is not None:
+            assert got == expect
+    # the subnormal-only case is a real subnormal maximum, not a flush to 0
+    assert oracle.amax_bf16(sub) > 0.0
+
+
 def test_rowfp8_matches_torch_cast():
     x = synth.normal_bf16((16, 384), 0.02, 1, 4)
     q, s = oracle.quant_rowwise_fp8(x)
