@@ -6,7 +6,10 @@
 // on which this file's device code is loaded reserves it until the process
 // exits.  Host code must not use the array's name as a device address (on
 // the host it names a host-side stand-in); its device address is looked up
-// once per device with cudaGetSymbolAddress and cached.
+// with cudaGetSymbolAddress on the first call made on each device and kept.
+// A cudaDeviceReset destroys the array with the context and leaves the kept
+// address stale, so a process that resets a device must not call this entry
+// point on that device afterwards.
 #include <mutex>
 
 #include "../../include/bsq.h"
@@ -22,25 +25,26 @@ constexpr size_t kScaleBytes = kMaxElems / 32 * sizeof(float);
 
 static __device__ __align__(256) unsigned char g_prefill_scratch[kCodeBytes + kScaleBytes];
 
-struct DeviceScratch {
-    std::once_flag once;
-    void *ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-};
 constexpr int kMaxDevices = 64;
-DeviceScratch g_devices[kMaxDevices];
+std::mutex g_lookup_mutex;
+void *g_device_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up on
-// the first call made with that device current).
+// Device address of the scratch array on the current device.  Only a
+// successful lookup is kept, so a lookup that failed (for example one made
+// during a stream capture) is simply tried again by the next call.
 cudaError_t scratch_on_current_device(void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    DeviceScratch &d = g_devices[dev];
-    std::call_once(d.once, [&d] { d.err = cudaGetSymbolAddress(&d.ptr, g_prefill_scratch); });
-    if (d.err != cudaSuccess) return d.err;
-    *out = d.ptr;
+    std::lock_guard<std::mutex> lock(g_lookup_mutex);
+    if (g_device_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_prefill_scratch);
+        if (e != cudaSuccess || p == nullptr) return e != cudaSuccess ? e : cudaErrorInvalidSymbol;
+        g_device_ptr[dev] = p;
+    }
+    *out = g_device_ptr[dev];
     return cudaSuccess;
 }
 
