@@ -5,12 +5,16 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - Tensor pointers are DEVICE pointers, allocated and owned by the caller.
- *    The library allocates no device memory and keeps no state beyond a
- *    launch counter and per-device attributes (SM count, kernel shared-
- *    memory limits) (the caller-owned-scratch convention of
- *    gemm_dense_int8.rs, `int8_gemm_faith2_prefill` doc comment, and of
- *    dispatch_proj_rowwise.rs, `cublas_fp8_rowwise_proj` doc comment).
+ *  - Tensor pointers are DEVICE pointers, allocated and owned by the caller
+ *    (the caller-owned-scratch convention of gemm_dense_int8.rs,
+ *    `int8_gemm_faith2_prefill` doc comment, and of dispatch_proj_rowwise.rs,
+ *    `cublas_fp8_rowwise_proj` doc comment).  The library allocates no device
+ *    memory at run time.  Its host state is a launch counter and per-device
+ *    caches (SM count, kernel attributes, one device address), each set
+ *    under a lock or atomically, so any host thread may call any entry
+ *    point.  The one piece of device memory it owns is the fixed scratch
+ *    array of int8_w4a8_prefill_noalloc (below), which every GPU that loads
+ *    the library's device code holds until the process exits.
  *  - BF16 tensors are passed as uint16_t bit patterns; E4M3 and packed E2M1
  *    as uint8_t.
  *  - Layouts are row-major with K innermost:
@@ -22,8 +26,9 @@
  *      outputs       BF16 [M, N]
  *  - The last argument is the CUDA stream (a cudaStream_t; NULL is the
  *    legacy default stream).  Every call is asynchronous and stream-ordered;
- *    no entry point synchronises the host (gemm_dense_int8.rs: "two launches
- *    on `stream` (stream-ordered)").
+ *    no entry point synchronises the host (gemm_dense_int8.rs,
+ *    `int8_gemm_faith2_prefill` doc comment: its launches are ordered on the
+ *    caller's stream).
  *  - Scalars (scale2, scaleA2, scaleB2) are host floats passed by value, as
  *    the pages pass them with `arg_f32`.
  *  - All scales are DEQUANT scales: value = code * scale.
@@ -33,7 +38,8 @@
  *    launches nothing.  Negative sizes are BSQ_ERR_INVALID_ARG.
  *  - Inputs must be finite.
  *  - Concurrent calls on different streams may run concurrently; they share
- *    no device memory.
+ *    no device memory, except calls of int8_w4a8_prefill_noalloc, which share
+ *    its scratch array and must not overlap on the GPU.
  *
  * Rounding: every quantised code and scale is defined bit-exactly (see each
  * function); GEMM and GEMV outputs are FP32 sums rounded once to BF16 and
@@ -108,6 +114,12 @@ BSQ_API bsq_status quantize_bf16_to_nvfp4(const uint16_t *in, uint8_t *packed,
  *   same FP32 round-to-nearest steps as the host form, so its codes and
  *   scales equal those of quantize_bf16_to_nvfp4 given that scale2.  An
  *   all-zero tensor (amax = 0) gets scale codes 0 and codes +0/-0.
+ *   The amax is only known on the device, so the scale2 checks of the host
+ *   form (finite, >= FLT_MIN) happen in the kernel: an amax that is NaN,
+ *   infinite, or non-zero but below 2688 * FLT_MIN makes the kernel write
+ *   scale2 = 0 and all-zero scales and codes (as for an all-zero tensor), so
+ *   w4a4_gemm_devscale then yields zeros, and sets bit 1 of the flags that
+ *   bsq_debug_take_timeouts returns.  The call itself still returns BSQ_OK.
  * Errors: as quantize_bf16_to_nvfp4; amax NULL -> INVALID_ARG.
  * ---------------------------------------------------------------------- */
 BSQ_API bsq_status quantize_bf16_to_nvfp4_devscale(const uint16_t *in, uint8_t *packed,
@@ -276,7 +288,10 @@ BSQ_API bsq_status int8_w4a8_prefill(const uint16_t *a_bf16, const int8_t *w_i8,
  * 41,943,040 activation elements.  Every GPU on which the library's device
  * code is loaded reserves it until the process exits.  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture.
+ * that device current; make that first call before any stream capture.  A
+ * lookup that fails returns BSQ_ERR_CUDA and is tried again by the next
+ * call; a successful one is kept for the life of the process, so do not call
+ * this entry point on a device after cudaDeviceReset.
  * This entry point allocates nothing and calls no allocating routine.
  * All calls share the array and it keeps the last call's contents; each
  * call writes every scratch byte it reads, so nothing needs clearing, but
@@ -294,8 +309,9 @@ BSQ_API bsq_status int8_w4a8_prefill_noalloc(const uint16_t *a_bf16, const int8_
  * requant_blockfp8_to_rowwise -- dispatch_proj_rowwise.rs,
  * `rowwise_pair_passthrough` and `requant_weight_rowwise_fp8_cached`.
  *   tag == BSQ_FP8_PER_ROW: *w_used = w, *scale_used = scale; nothing is
- *     launched and nothing is written (the "passes through verbatim"
- *     invariant of that page's tests).  w_out/scale_out may be NULL.
+ *     launched and nothing is written (the invariant that page's unit tests
+ *     check: a row-wise weight comes back unchanged, with no conversion).
+ *     w_out/scale_out may be NULL.
  *   tag == BSQ_FP8_BLOCK_SCALED: w E4M3 [n, k] with scale FP32
  *     [n/128, k/128] -> w_out E4M3 [n, k] + scale_out FP32 [n]; then
  *     *w_used = w_out, *scale_used = scale_out.  Per element the BF16
@@ -346,11 +362,12 @@ BSQ_API const char *bsq_status_string(bsq_status status);
  * nothing (the passthrough) or count the launches of a timed region. */
 BSQ_API uint64_t bsq_debug_launch_count(void);
 
-/* Synchronises the current device, then returns and clears the flags that
- * the tensor-core kernels set when one of their bounded waits ran out (0 when
- * none did; 0xFFFFFFFF when the device could not be read).  For tests and
- * debugging: every wait inside a libbsq kernel gives up after 2 s instead of
- * hanging, and records it here. */
+/* Synchronises the current device, then returns and clears the flags the
+ * kernels set on the device (0 when none was set; 0xFFFFFFFF when the device
+ * could not be read).  Bit 0: one of their bounded waits ran out -- every
+ * wait inside a libbsq kernel gives up after 2 s instead of hanging, and
+ * records it here.  Bit 1: quantize_bf16_to_nvfp4_devscale met an amax whose
+ * scale2 the host form rejects.  For tests and debugging. */
 BSQ_API uint32_t bsq_debug_take_timeouts(void);
 
 #ifdef __cplusplus

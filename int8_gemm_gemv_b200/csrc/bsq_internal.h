@@ -6,7 +6,37 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 namespace bsq {
+
+constexpr int kMaxDevices = 64;
+
+// Runs a per-device set-up step (kernel attributes) once per device, with
+// that device current, keeping only a success.  Any host thread may call
+// it: concurrent first calls serialise on the mutex, later ones read one
+// atomic flag.  Devices past kMaxDevices run the step on every call.
+class DeviceOnce {
+  public:
+    template <class F>
+    cudaError_t run(F &&init) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDevices) return init();
+        if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        e = init();
+        if (e == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+        return e;
+    }
+
+  private:
+    std::atomic<bool> done_[kMaxDevices] = {};
+    std::mutex mu_;
+};
 
 // Count of kernels launched by the library (bsq_debug_launch_count).
 void note_launch();

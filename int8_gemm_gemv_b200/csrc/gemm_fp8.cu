@@ -207,15 +207,11 @@ cudaError_t launch_fp8_gemm_rowscale(const uint8_t *a, const float *a_scale, con
     if (!make_tmap_2d(&tA, a, 1, k, m, k, BK, BM, true, false) ||
         !make_tmap_2d(&tB, w, 1, k, n, k, BK, BN, true, false))
         return cudaErrorInvalidValue;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(k_fp8_gemm_rowscale, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+    static DeviceOnce attrs;
+    cudaError_t e = attrs.run([] {
+        return cudaFuncSetAttribute(k_fp8_gemm_rowscale, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
     const int tiles = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
     k_fp8_gemm_rowscale<<<grid, kThreads, kSmemBytes, s>>>(tA, tB, a_scale, w_scale, out, m, n, k);

@@ -349,20 +349,17 @@ cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const
         !make_tmap_2d(&tSA, a_scale, 4, kblk, m, kblk * 4, 4, BM, false, true) ||
         !make_tmap_2d(&tSW, w_scale, 4, kblk, n, kblk * 4, 4, BN, false, true))
         return cudaErrorInvalidValue;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
+    static DeviceOnce attrs;
+    cudaError_t e = attrs.run([] {
         // The register split is only valid for a block launched with exactly
         // kLaunchRegs registers per thread.
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, k_int8_gemm);
-        if (e != cudaSuccess) return e;
+        cudaError_t r = cudaFuncGetAttributes(&fa, k_int8_gemm);
+        if (r != cudaSuccess) return r;
         if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-        e = cudaFuncSetAttribute(k_int8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+        return cudaFuncSetAttribute(k_int8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
     const int tiles = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
     k_int8_gemm<<<grid, kThreads, kSmemBytes, s>>>(tA, tB, tSA, tSW, out, m, n, k);

@@ -367,14 +367,19 @@ uint32_t take_timeouts_gemm_w4a4() {
 
 // CTA pairs that can be resident at once (cached per device).
 static int w4a4_max_pairs(cudaLaunchConfig_t cfg) {
-    static int cached[64] = {};
+    // a racing first call computes the same value twice; the store is atomic
+    static std::atomic<int> cached[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    const bool cacheable = dev >= 0 && dev < kMaxDevices;
+    if (cacheable) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     cfg.gridDim = dim3(sm_count());
     if (cudaOccupancyMaxActiveClusters(&n, k_w4a4_gemm, &cfg) != cudaSuccess || n <= 0) n = sm_count() / 2;
-    if (dev >= 0 && dev < 64) cached[dev] = n;
+    if (cacheable) cached[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
@@ -394,14 +399,11 @@ cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, co
         !make_tmap_2d(&tSA, a_scale, 1, ks, m, ks, 16, BM, false, false) ||
         !make_tmap_2d(&tSB, w_scale, 1, ks, n, ks, 16, BN, false, false))
         return cudaErrorInvalidValue;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_w4a4_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+    static DeviceOnce attrs;
+    cudaError_t e = attrs.run([] {
+        return cudaFuncSetAttribute(k_w4a4_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    });
+    if (e != cudaSuccess) return e;
     const int tiles = ((m + 2 * BM - 1) / (2 * BM)) * ((n + BN - 1) / BN);
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreads);
@@ -422,7 +424,7 @@ cudaError_t launch_w4a4_gemm(const uint8_t *a_packed, const uint8_t *a_scale, co
     cfg.numAttrs = 2;
     const int pairs = tiles < max_pairs ? tiles : max_pairs;
     cfg.gridDim = dim3(2 * pairs);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, k_w4a4_gemm, tA, tB, tSA, tSB, tO, use_tma_store, out, scale_ab,
+    e = cudaLaunchKernelEx(&cfg, k_w4a4_gemm, tA, tB, tSA, tSB, tO, use_tma_store, out, scale_ab,
                                        scale_b_dev, m, n, k);
     note_launch();
     return e;

@@ -320,15 +320,12 @@ cudaError_t launch_na(const uint8_t *a_packed, const uint8_t *a_scale, const uin
         !make_tmap_2d(&tSA, a_scale, 1, ks, m, ks, 16, ma, false, false) ||
         !make_tmap_2d(&tSW, w_scale, 1, ks, n, ks, 16, BW, false, false))
         return cudaErrorInvalidValue;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(k_w4a4_small<NA>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes<NA>());
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+    static DeviceOnce attrs;
+    cudaError_t e = attrs.run([] {
+        return cudaFuncSetAttribute(k_w4a4_small<NA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem_bytes<NA>());
+    });
+    if (e != cudaSuccess) return e;
     const int tiles = (n + BW - 1) / BW;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles < sm_count() ? tiles : sm_count());

@@ -41,17 +41,12 @@ namespace bsq {
 
 namespace {
 
-#ifndef BSQ_GEMV_CONSUMERS
-#define BSQ_GEMV_CONSUMERS 16
-#define BSQ_GEMV_KS 1024
-#define BSQ_GEMV_STAGES 6
-#endif
-constexpr int kConsumers = BSQ_GEMV_CONSUMERS;
+constexpr int kConsumers = 16;
 constexpr int kThreads = 32 * (kConsumers + 1);
-constexpr int KS = BSQ_GEMV_KS;              // K bytes per stage (64 per consumer warp)
+constexpr int KS = 1024;                     // K bytes per stage (64 per consumer warp)
 constexpr int TILE_BYTES = 16 * KS;          // 16 KB: 16 rows x 1024 B
 constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // two tiles
-constexpr int STAGES = BSQ_GEMV_STAGES;      // ring of STAGES x 2 tiles
+constexpr int STAGES = 6;                    // ring of STAGES x 2 tiles
 constexpr int BOX = 128;                     // TMA box: 128 B x 16 rows
 constexpr uint64_t kPrefetchBytes = 256 << 10;  // per CTA, before the stream dependency
 
@@ -350,15 +345,12 @@ template <int MT, bool BS>
 static cudaError_t launch_mt(const CUtensorMap &tm, const CUtensorMap &tm8, int tm3d, const uint8_t *w,
                              const uint16_t *in, const float *row_scale, uint16_t *out, int m, int n, int k,
                              cudaStream_t s) {
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_fp8_gemv<MT, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem_bytes<MT>());
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+    static DeviceOnce attrs;
+    cudaError_t e = attrs.run([] {
+        return cudaFuncSetAttribute(k_fp8_gemv<MT, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem_bytes<MT>());
+    });
+    if (e != cudaSuccess) return e;
     const int units = (n + 7) / 8;
     const int grid = units < sm_count() ? units : sm_count();
     cudaLaunchConfig_t cfg = {};

@@ -16,6 +16,8 @@
 // are not divided out one by one: a bracket of two products decides the code
 // and the exact division runs only where the bracket straddles a rounding
 // boundary (see `Bracket`).
+#include <cfloat>
+
 #include "bsq_common.cuh"
 
 namespace bsq {
@@ -24,10 +26,12 @@ namespace {
 
 // Grid-stride quantisers take this many independent units per thread and
 // pass, so several loads per thread are in flight at once.
-#ifndef BSQ_QUANT_UNROLL
-#define BSQ_QUANT_UNROLL 2
-#endif
-constexpr int kQuantUnroll = BSQ_QUANT_UNROLL;
+constexpr int kQuantUnroll = 2;
+
+// Flags of this file's kernels, read and cleared by take_timeouts_quant: bit
+// 0, a bounded wait of the bulk-copy requant ran out; bit 1, the device-
+// scale2 NVFP4 quantiser met an amax whose scale2 the host form rejects.
+static __device__ unsigned int g_quant_timeouts;
 
 __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
     uint4 r;
@@ -236,10 +240,21 @@ __global__ void __launch_bounds__(256) k_quant_nvfp4(const uint4 *__restrict__ i
     // serialization may start its prologue now; it reads these outputs only
     // after griddepcontrol.wait, i.e. after this grid has completed
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    bool zero_all = false;
     if (amax_dev != nullptr) {
         // the weight's scale2 from its device amax, the same FP32 steps as
         // on the host: scale2 = amax / (6 * 448), t6 = 6 * scale2
-        scale2 = __fdiv_rn(__ldg(amax_dev), 2688.0f);
+        const float amax = __ldg(amax_dev);
+        scale2 = __fdiv_rn(amax, 2688.0f);
+        // The host form accepts only a finite scale2 >= FLT_MIN.  A scale2 it
+        // would reject (an amax that is NaN, infinite, or below 2688 *
+        // FLT_MIN but not 0) gives what an all-zero tensor gives -- scale2
+        // 0, every scale and code 0 -- and sets flag bit 1.
+        if (amax != 0.0f && !(scale2 >= FLT_MIN && scale2 <= FLT_MAX)) {
+            zero_all = true;
+            scale2 = 0.0f;
+            if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(&g_quant_timeouts, 2u);
+        }
         t6 = __fmul_rn(6.0f, scale2);
         if (scale2_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *scale2_out = scale2;
     }
@@ -264,7 +279,8 @@ __global__ void __launch_bounds__(256) k_quant_nvfp4(const uint4 *__restrict__ i
             const uint32_t mx = max(amax_bits_8(v[u][0]), amax_bits_8(v[u][1]));
             // an all-zero block has scale code 0 (also when scale2 is 0: an
             // all-zero tensor's device amax)
-            const uint8_t sc = mx == 0 ? (uint8_t)0 : e4m3_of_quotient(__uint_as_float(mx << 16), t6, t6b);
+            const uint8_t sc =
+                (mx == 0 || zero_all) ? (uint8_t)0 : e4m3_of_quotient(__uint_as_float(mx << 16), t6, t6b);
             const float sfv = e4m3_to_f32(sc);
             uint2 codes = make_uint2(0u, 0u);
             if (sfv != 0.0f) {
@@ -358,14 +374,8 @@ __device__ __forceinline__ uint32_t cta_max_once(uint32_t v, uint32_t *red) {
 // with the row's 16-byte chunks kept in registers (kRowKeep per thread, so
 // rows of up to kRowThreads * kRowKeep * 8 elements; longer rows are read
 // again in pass 2), pass 2 writes the codes.
-#ifndef BSQ_ROW_THREADS
-#define BSQ_ROW_THREADS 128
-#endif
-#ifndef BSQ_ROW_KEEP
-#define BSQ_ROW_KEEP 5
-#endif
-constexpr int kRowThreads = BSQ_ROW_THREADS;
-constexpr int kRowKeep = BSQ_ROW_KEEP;
+constexpr int kRowThreads = 128;
+constexpr int kRowKeep = 5;
 
 __global__ void __launch_bounds__(kRowThreads) k_quant_rowwise_fp8(const uint16_t *__restrict__ in,
                                                                    uint8_t *__restrict__ q,
@@ -460,14 +470,8 @@ __device__ __forceinline__ uint4 requant_codes_16(const Bf16x16 &t, float s, con
 
 // One CTA of kReqThreads per row, the row's transients kept in registers
 // (kReqKeep chunks per thread; longer rows are dequantised again).
-#ifndef BSQ_REQ_THREADS
-#define BSQ_REQ_THREADS 256
-#endif
-#ifndef BSQ_REQ_KEEP
-#define BSQ_REQ_KEEP 2
-#endif
-constexpr int kReqThreads = BSQ_REQ_THREADS;
-constexpr int kReqKeep = BSQ_REQ_KEEP;
+constexpr int kReqThreads = 256;
+constexpr int kReqKeep = 2;
 
 __global__ void __launch_bounds__(kReqThreads) k_requant_blockfp8_to_rowwise(const uint8_t *__restrict__ w,
                                                                              const float *__restrict__ bscale,
@@ -515,8 +519,6 @@ __global__ void __launch_bounds__(kReqThreads) k_requant_blockfp8_to_rowwise(con
 // memory.
 constexpr int kReqRowThreads = 64;
 constexpr int kReqSmemMaxK = 48 * 1024;
-
-static __device__ unsigned int g_quant_timeouts;
 
 __global__ void __launch_bounds__(kReqRowThreads) k_requant_blockfp8_rows_smem(const uint8_t *__restrict__ w,
                                                                               const float *__restrict__ bscale,

@@ -60,14 +60,19 @@ bool make_tmap_rows_chunks(void *tmap_out, const void *base, uint64_t k_bytes, u
 }
 
 int sm_count() {
-    static int cached[64] = {};
+    // a racing first call computes the same value twice; the store is atomic
+    static std::atomic<int> cached[kMaxDevices];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    const bool cacheable = dev >= 0 && dev < kMaxDevices;
+    if (cacheable) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (n <= 0) n = 148;
-    if (dev >= 0 && dev < 64) cached[dev] = n;
+    if (cacheable) cached[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 

@@ -1,6 +1,6 @@
 """Run one libbsq kernel a few times at a given shape, for profiler captures.
 
-    python -m int8_gemm_gemv_b200.profile_case w4a4 --m 4096 --n 17408 --k 5120 --iters 3
+    python profile_case.py w4a4 --m 4096 --n 17408 --k 5120 --iters 3
 
 Inputs are random codes in device memory (the kernel's cost does not depend
 on their values beyond power); nothing is checked.  Kinds: w4a4 (M <= 128
@@ -10,8 +10,12 @@ quant_nvfp4, quant_rowfp8, quant_int8, requant_w, requant_block.
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import torch
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
 import int8_gemm_gemv_b200 as bsq
 

@@ -125,6 +125,30 @@ def test_nvfp4_device_scale2_all_zero():
     assert float(s2.item()) == 0.0 and not host(p).any() and not host(sf).any()
 
 
+@pytest.mark.parametrize("amax", [float("nan"), float("inf"), 1e-36])
+def test_nvfp4_device_scale2_rejected_amax(amax):
+    """An amax whose scale2 (amax / 2688) the host form rejects -- NaN,
+    infinite, or non-zero below 2688 * FLT_MIN -- quantises like an all-zero
+    tensor (scale2 0, zero scales and codes), the GEMM then gives zeros, and
+    flag bit 1 is raised once."""
+    m, n, k = 16, 64, 256
+    x = synth.normal_bf16((n, k), 0.02, 0, 8)
+    xd = to_dev(x)
+    amax_dev = torch.tensor([amax], dtype=torch.float32, device="cuda")
+    p = torch.full((n, k // 2), 0x55, dtype=torch.uint8, device="cuda")
+    sf = torch.full((n, k // 16), 0x55, dtype=torch.uint8, device="cuda")
+    s2 = torch.full((1,), 1.0, dtype=torch.float32, device="cuda")
+    bsq.quantize_bf16_to_nvfp4_devscale(xd, p, sf, amax_dev, s2, n, k)
+    torch.cuda.synchronize()
+    assert float(s2.item()) == 0.0 and not host(p).any() and not host(sf).any()
+    assert bsq.debug_take_timeouts() == 2
+    ap, asf = oracle.quant_nvfp4(synth.normal_bf16((m, k), 1.0, 0, 9), 1.0)
+    out = bf16_out((m, n))
+    bsq.w4a4_gemm_devscale(to_dev(ap), to_dev(asf), p, sf, out, 1.0, s2, m, n, k)
+    torch.cuda.synchronize()
+    assert np.all(oracle.bf16_to_f32(host(out, np.uint16)) == 0.0)
+
+
 def test_w4a4_structured_one_hot():
     """One-hot activation rows pick single weight elements: checks nibble
     order, scale placement per row and per 16-block, and the M/N tiling."""
