@@ -170,8 +170,12 @@ BSQ_API bsq_status w4a4_gemm_devscale(const uint8_t *a_packed, const uint8_t *a_
  *   row_scale FP32 [n]          per-row dequant scale, applied at write-out
  *   out       BF16 [m, n]
  *   out[i,j] = row_scale[j] * sum_k bf16(in[i,k]) * e4m3(w[j,k])
- * The sum for one output does not depend on m (a row computed alone or in a
- * batch of 16 gives the same bits).
+ * FP32 sums, one BF16 rounding.  Inside, each activation row is scaled by a
+ * power of two and run through FP16 tensor-core MMAs: products are exact for
+ * every activation within 2^31 of its row's largest magnitude; smaller ones
+ * are rounded, each by less than 2^-39 of that magnitude.  The sum for one
+ * output does not depend on m (a row computed alone or in a batch of 16
+ * gives the same bits).
  * Errors: m outside 1..16 -> INVALID_ARG; k % 16 != 0 -> INVALID_ARG
  * (both as the page's launchers reject them).
  * ---------------------------------------------------------------------- */
@@ -189,8 +193,8 @@ BSQ_API bsq_status fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w,
  *   out         BF16 [m, n]
  *   out[i,j] = sum_k bf16(in[i,k]) * e4m3(w[j,k]) * block_scale[j/128, k/128]
  * FP32 sums per 64-wide K chunk, scaled by their block and accumulated in
- * FP32; one BF16 rounding.  As for fp8_gemv_rowscale, an output does not
- * depend on m.
+ * FP32; one BF16 rounding.  The same FP16 datapath and exactness condition
+ * as fp8_gemv_rowscale; an output does not depend on m.
  * Errors: m outside 1..16 or k % 16 != 0 -> INVALID_ARG; n or k not a
  * multiple of 128 -> UNSUPPORTED (the block grid needs whole blocks).
  * ---------------------------------------------------------------------- */
@@ -354,6 +358,21 @@ BSQ_API bsq_status fp8_gemm_rowscale(const uint8_t *a, const float *a_scale,
 BSQ_API bsq_status bsq_amax_bf16(const uint16_t *x, size_t count, float *amax_dev,
                          bsq_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * bsq_debug_stream_read -- a kernel that only reads `bytes` bytes at `src`
+ * (16-byte aligned, a multiple of 16 bytes) and XORs one word per CTA into
+ * *sink (device, 4-byte aligned): the HBM streaming floor that the
+ * bandwidth-bound kernels are measured against.  It is launched like the
+ * FP8 GEMV (one CTA per SM, programmatic stream serialization).  mode 0: a
+ * 128 KB ring of bulk copies per CTA; mode 1: as the GEMV does for
+ * consecutive launches, each CTA prefetches its share into L2 before the
+ * stream dependency and uses a 64 KB ring, so two launches can overlap.
+ * No counterpart on the pages (a measurement aid).
+ * Errors: mode not 0 or 1, bytes % 16 != 0 -> INVALID_ARG.
+ * ---------------------------------------------------------------------- */
+BSQ_API bsq_status bsq_debug_stream_read(const void *src, size_t bytes, uint32_t *sink, int mode,
+                                         bsq_stream_t stream);
+
 /* Text of a status code (static storage). */
 BSQ_API const char *bsq_status_string(bsq_status status);
 
@@ -361,6 +380,13 @@ BSQ_API const char *bsq_status_string(bsq_status status);
  * devices, all threads).  Lets a caller or test check that a call launched
  * nothing (the passthrough) or count the launches of a timed region. */
 BSQ_API uint64_t bsq_debug_launch_count(void);
+
+/* The CUDA error code (a cudaError_t value) behind the last BSQ_ERR_CUDA
+ * that an entry point returned on the calling thread, and clears it (0 when
+ * there was none).  bsq_debug_cuda_error_string gives its text (static
+ * storage). */
+BSQ_API int bsq_debug_take_cuda_error(void);
+BSQ_API const char *bsq_debug_cuda_error_string(int code);
 
 /* Synchronises the current device, then returns and clears the flags the
  * kernels set on the device (0 when none was set; 0xFFFFFFFF when the device

@@ -35,9 +35,10 @@ def library_path() -> str:
 
 
 class BsqError(RuntimeError):
-    def __init__(self, status: int, fn: str):
+    def __init__(self, status: int, fn: str, detail: str | None = None):
         self.status = status
-        super().__init__(f"{fn}: {status_string(status)}")
+        msg = f"{fn}: {status_string(status)}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
 
 
 _lib = None
@@ -62,6 +63,7 @@ _SIGS = {
     "requant_blockfp8_to_rowwise": [_I, _P, _P, _I, _I, _P, _P, ctypes.POINTER(_P), ctypes.POINTER(_P), _P],
     "fp8_gemm_rowscale": [_P, _P, _P, _P, _P, _I, _I, _I, _P],
     "bsq_amax_bf16": [_P, ctypes.c_size_t, _P, _P],
+    "bsq_debug_stream_read": [_P, ctypes.c_size_t, _P, _I, _P],
 }
 
 
@@ -84,6 +86,10 @@ def lib() -> ctypes.CDLL:
         L.bsq_debug_launch_count.restype = ctypes.c_uint64
         L.bsq_debug_take_timeouts.argtypes = []
         L.bsq_debug_take_timeouts.restype = ctypes.c_uint32
+        L.bsq_debug_take_cuda_error.argtypes = []
+        L.bsq_debug_take_cuda_error.restype = ctypes.c_int
+        L.bsq_debug_cuda_error_string.argtypes = [ctypes.c_int]
+        L.bsq_debug_cuda_error_string.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -110,9 +116,14 @@ def _stream(stream):
 
 
 def _call(name, *args):
-    st = getattr(lib(), name)(*args)
+    L = lib()
+    st = getattr(L, name)(*args)
     if st != BSQ_OK:
-        raise BsqError(st, name)
+        detail = None
+        if st == BSQ_ERR_CUDA:
+            code = L.bsq_debug_take_cuda_error()
+            detail = f"cudaError {code}: {L.bsq_debug_cuda_error_string(code).decode()}"
+        raise BsqError(st, name, detail)
 
 
 def status_string(status: int) -> str:
@@ -204,3 +215,8 @@ def fp8_gemm_rowscale(a, a_scale, w, w_scale, out, m, n, k, stream=None):
 
 def bsq_amax_bf16(x, count, amax_dev, stream=None):
     _call("bsq_amax_bf16", _ptr(x), count, _ptr(amax_dev), _stream(stream))
+
+
+def debug_stream_read(src, nbytes, sink, mode=0, stream=None):
+    """Read-only streaming kernel over nbytes of src (the HBM floor)."""
+    _call("bsq_debug_stream_read", _ptr(src), nbytes, _ptr(sink), mode, _stream(stream))

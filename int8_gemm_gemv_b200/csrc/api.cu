@@ -11,13 +11,22 @@
 namespace bsq {
 static std::atomic<uint64_t> g_launches{0};
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+// the CUDA error behind the calling thread's last BSQ_ERR_CUDA
+static thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+void note_cuda_error(cudaError_t e) {
+    if (e != cudaSuccess) t_last_cuda_error = e;
+}
 }  // namespace bsq
 
 namespace {
 
 inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
-inline bsq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BSQ_OK : BSQ_ERR_CUDA; }
+inline bsq_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return BSQ_OK;
+    bsq::note_cuda_error(e);
+    return BSQ_ERR_CUDA;
+}
 inline cudaStream_t cs(bsq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 // scale2 divides and multiplies block scales: a finite, positive, normal float
 inline bool valid_scale2(float s) { return std::isfinite(s) && s >= FLT_MIN; }
@@ -169,7 +178,7 @@ bsq_status int8_w4a8_prefill(const uint16_t *a_bf16, const int8_t *w_i8, const f
     st = check_int8_gemm(a_i8_scratch, w_i8, a_scale_scratch, w_scale, out, m, n, k);
     if (st != BSQ_OK || m == 0 || n == 0) return st;
     cudaError_t e = bsq::launch_quant_act_int8_per32(a_bf16, a_i8_scratch, a_scale_scratch, m, k, cs(stream));
-    if (e != cudaSuccess) return BSQ_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
     return cuda_status(
         bsq::launch_int8_blockscaled_gemm(a_i8_scratch, w_i8, a_scale_scratch, w_scale, out, m, n, k, cs(stream)));
 }
@@ -200,7 +209,7 @@ bsq_status requant_blockfp8_to_rowwise(bsq_format tag, const uint8_t *w, const f
     if (!al16(w) || !al16(w_out) || !al4(scale) || !al4(scale_out)) return BSQ_ERR_MISALIGNED;
     if (n > 0) {
         cudaError_t e = bsq::launch_requant_blockfp8_to_rowwise(w, scale, n, k, w_out, scale_out, cs(stream));
-        if (e != cudaSuccess) return BSQ_ERR_CUDA;
+        if (e != cudaSuccess) return cuda_status(e);
     }
     *w_used = w_out;
     *scale_used = scale_out;
@@ -223,6 +232,14 @@ bsq_status bsq_amax_bf16(const uint16_t *x, size_t count, float *amax_dev, bsq_s
     return cuda_status(bsq::launch_amax_bf16(x, count, amax_dev, cs(stream)));
 }
 
+bsq_status bsq_debug_stream_read(const void *src, size_t bytes, uint32_t *sink, int mode, bsq_stream_t stream) {
+    if ((mode != 0 && mode != 1) || bytes % 16) return BSQ_ERR_INVALID_ARG;
+    if (bytes == 0) return BSQ_OK;
+    if (!src || !sink) return BSQ_ERR_INVALID_ARG;
+    if (!al16(src) || !al4(sink)) return BSQ_ERR_MISALIGNED;
+    return cuda_status(bsq::launch_stream_read(src, bytes, sink, mode, cs(stream)));
+}
+
 const char *bsq_status_string(bsq_status status) {
     switch (status) {
         case BSQ_OK: return "BSQ_OK";
@@ -236,10 +253,19 @@ const char *bsq_status_string(bsq_status status) {
 
 uint64_t bsq_debug_launch_count(void) { return bsq::g_launches.load(std::memory_order_relaxed); }
 
+int bsq_debug_take_cuda_error(void) {
+    const cudaError_t e = bsq::t_last_cuda_error;
+    bsq::t_last_cuda_error = cudaSuccess;
+    return (int)e;
+}
+
+const char *bsq_debug_cuda_error_string(int code) { return cudaGetErrorString((cudaError_t)code); }
+
 uint32_t bsq_debug_take_timeouts(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return 0xFFFFFFFFu;
     return bsq::take_timeouts_gemm_w4a4() | bsq::take_timeouts_gemm_w4a4_small() | bsq::take_timeouts_gemm_fp8() |
-           bsq::take_timeouts_gemm_int8() | bsq::take_timeouts_gemv() | bsq::take_timeouts_quant();
+           bsq::take_timeouts_gemm_int8() | bsq::take_timeouts_gemv() | bsq::take_timeouts_quant() |
+           bsq::take_timeouts_stream_read();
 }
 
 }  // extern "C"

@@ -40,6 +40,9 @@ class DeviceOnce {
 
 // Count of kernels launched by the library (bsq_debug_launch_count).
 void note_launch();
+// Records the CUDA error behind a BSQ_ERR_CUDA for the calling thread
+// (bsq_debug_take_cuda_error).
+void note_cuda_error(cudaError_t e);
 
 // Per-file flags of bounded waits that ran out (read and cleared with a
 // device synchronisation; used by tests only).
@@ -49,6 +52,7 @@ uint32_t take_timeouts_gemm_w4a4_small();
 uint32_t take_timeouts_gemm_fp8();
 uint32_t take_timeouts_gemm_int8();
 uint32_t take_timeouts_gemv();
+uint32_t take_timeouts_stream_read();
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
@@ -68,6 +72,11 @@ cudaError_t launch_requant_w_nvfp4_int8(const uint8_t *packed, const uint8_t *sf
 cudaError_t launch_quant_act_int8_per32(const uint16_t *a, int8_t *q, float *scale, int m, int k,
                                         cudaStream_t s);
 cudaError_t launch_amax_bf16(const uint16_t *x, size_t count, float *amax, cudaStream_t s);
+
+// ---- launchers (stream_read.cu) ----
+// mode 0: one CTA per SM, 128 KB ring; mode 1: L2 prefetch of each CTA's
+// share before the stream dependency and a 64 KB ring (two CTAs per SM)
+cudaError_t launch_stream_read(const void *src, uint64_t bytes, uint32_t *sink, int mode, cudaStream_t s);
 
 // ---- launchers (gemv_fp8.cu) ----
 cudaError_t launch_fp8_gemv_rowscale(const uint16_t *in, const uint8_t *w, const float *row_scale, uint16_t *out,
@@ -98,6 +107,13 @@ struct CUtensorMap_st_holder;
 bool make_tmap_2d(void *tmap_out, const void *base, int elem_bytes, uint64_t cols, uint64_t rows,
                   uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128,
                   bool elem_is_float);
+
+// General tiled tensor map: `rank` dimensions (innermost first) of `dims`
+// elements of elem_bytes bytes, `strides` (rank - 1 byte strides of dims 1..),
+// box `box`, swizzle of 0, 32, 64 or 128 bytes.  Out-of-range box elements
+// are zero-filled on load.
+bool make_tmap(void *tmap_out, const void *base, int elem_bytes, int rank, const uint64_t *dims,
+               const uint64_t *strides, const uint32_t *box, int swizzle_bytes);
 
 // 3-D view of a row-major [rows, k_bytes] byte matrix as (128 B, rows,
 // k_bytes/128 chunks) so one TMA copy moves box_rows x (box_chunks * 128 B)

@@ -214,6 +214,28 @@ def test_gemv_cfg2(gemv_weight, m):
     check_tol(g, ob, ab, f"gemv m={m}")
 
 
+def test_gemv_activation_range(gemv_weight):
+    """The GEMV runs its activations through FP16 with a per-row power of two,
+    so rows far from 1 in magnitude must still match the oracle: a row
+    scaled by 2^100, one by 2^-100, an all-zero row, and a row whose largest
+    element is 2^20 times its others; each row's result must also equal the
+    same row computed alone (the scale is per row)."""
+    wq, ws = gemv_weight
+    base = synth.normal_bf16((4, 5120), 1.0, 2, 7)
+    x = oracle.bf16_to_f32(base).astype(np.float32)
+    x[0] *= np.float32(2.0**100)
+    x[1] *= np.float32(2.0**-100)
+    x[2] = 0.0
+    x[3, 17] = np.float32(2.0**20)
+    inp = synth.to_bf16_bits(x)
+    g = run_gemv(inp, wq, ws)
+    ob, _, ab = oracle.fp8_gemv_rowscale(inp, wq, ws)
+    check_tol(g, ob, ab, "gemv activation range")
+    assert np.all(oracle.bf16_to_f32(g[2]) == 0.0)
+    for r in range(4):
+        assert np.array_equal(run_gemv(inp[r:r + 1].copy(), wq, ws), g[r:r + 1]), r
+
+
 def test_gemv_row_independent_of_batch(gemv_weight):
     """A row computed alone, or in a batch of 2, 8 or 16, gives the same bits
     (fp8_gemv_batch.rs: the batched kernels are bit-identical per row)."""
@@ -264,6 +286,61 @@ def test_gemv_blockscaled_row_independent_of_batch():
     for m in (1, 4):
         part = run_gemv_bs(inp[:m].copy(), wq, S)
         assert np.array_equal(part, all16[:m])
+
+
+# lm_head-sized N: many tile groups per CTA, ragged N, K % 64 != 0 (one copy
+# per 64-byte chunk) and K % 64 == 0 (one copy per slot)
+@pytest.mark.parametrize("nkm", [(75781, 80, 1), (75781, 80, 9), (80000, 128, 2), (80000, 128, 16)])
+def test_gemv_large_n_ragged(nkm):
+    n, k, m = nkm
+    inp, w_bf = synth.gemv_inputs(m, n, k, seed=9)
+    wq, ws = oracle.quant_rowwise_fp8(w_bf)
+    g = run_gemv(inp, wq, ws)
+    ob, _, ab = oracle.fp8_gemv_rowscale(inp, wq, ws)
+    check_tol(g, ob, ab, f"gemv large n {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("n", [256, 76800])
+def test_gemv_every_code_exact(n):
+    """Every finite E4M3 byte, each picked out by a one-hot activation row
+    with row scale 1: the output is the code's value, exact in BF16, so the
+    E4M3 conversion inside the kernel must match the oracle bit for bit
+    (one tile group per CTA at n = 256, many at n = 76800)."""
+    k, m = 256, 16
+    codes = np.arange(256, dtype=np.uint8)
+    codes[codes == 0x7F] = 0x7E
+    codes[codes == 0xFF] = 0xFE
+    wq = np.empty((n, k), np.uint8)
+    for r in range(n):  # a different rotation per row, so every code meets every one-hot column
+        wq[r] = np.roll(codes, r % 256)
+    ws = np.ones(n, np.float32)
+    inp = np.zeros((m, k), np.uint16)
+    hot = np.random.default_rng(3).choice(k, m, replace=False)
+    inp[np.arange(m), hot] = 0x3F80  # 1.0
+    g = run_gemv(inp, wq, ws)
+    ob, _, _ = oracle.fp8_gemv_rowscale(inp, wq, ws)
+    assert np.array_equal(g, ob)
+
+
+@pytest.mark.parametrize("mn", [(3, 76800), (11, 76800)])
+def test_gemv_blockscaled_large_n(mn):
+    m, n = mn
+    k = 256
+    inp, w_bf = synth.gemv_inputs(m, n, k, seed=10)
+    wq, S = oracle.quant_blockfp8(w_bf)
+    g = run_gemv_bs(inp, wq, S)
+    ob, _, ab = oracle.fp8_gemv_blockscaled(inp, wq, S)
+    check_tol(g, ob, ab, f"gemv block-scaled large n {m}x{n}x{k}")
+
+
+def test_gemv_large_n_independent_of_batch():
+    n, k = 76800, 512
+    inp, w_bf = synth.gemv_inputs(16, n, k, seed=11)
+    wq, ws = oracle.quant_rowwise_fp8(w_bf)
+    full = run_gemv(inp, wq, ws)
+    for m in (1, 8, 9):
+        part = run_gemv(inp[:m].copy(), wq, ws)
+        assert np.array_equal(part, full[:m]), m
 
 
 def test_gemv_lm_head_shape():
