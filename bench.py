@@ -386,6 +386,18 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
             bsq.quant_rowwise_fp8(src, wq, ws, n, k, stream)
             return wq, ws
         ws_list = rotate(mk_w, n * k)
+        # the floor: a read-only kernel launched like the GEMV (one CTA per SM,
+        # programmatic stream serialization) over the same rotating copies
+        sink = torch.zeros(1, dtype=torch.int32, device=dev)
+        itf = [0]
+
+        def floor_fn(st):
+            wq, _ = ws_list[itf[0] % len(ws_list)]
+            itf[0] += 1
+            bsq.debug_stream_read(wq, n * k, sink, 0, st)
+        t_floor = time_graph(torch, floor_fn, 4 * len(ws_list))
+        hbm_row(f"floor_stream_read_{n}x{k}", t_floor, n * k,
+                {"l2": f"{len(ws_list)} rotating weight copies", "kernel": "bsq_debug_stream_read (read only)"})
         for m in ms:
             x = bf16_rand((m, k), 1.0)
             out = torch.empty((m, n), dtype=torch.int16, device=dev)
@@ -397,7 +409,8 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
                 bsq.fp8_gemv_rowscale(x, wq, ws, out, m, n, k, st)
             t = time_graph(torch, f, 4 * len(ws_list))
             hbm_row(f"a4_fp8_gemv_m{m}_n{n}_k{k}", t, n * k + 4 * n + 2 * m * k + 2 * m * n,
-                    {"l2": f"{len(ws_list)} rotating weight copies"})
+                    {"l2": f"{len(ws_list)} rotating weight copies",
+                     "frac_of_stream_read_floor": round(t_floor / t, 4)})
         del ws_list
         torch.cuda.empty_cache()
 
