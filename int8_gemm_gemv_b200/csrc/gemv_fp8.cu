@@ -10,9 +10,11 @@
 //
 // The weight stream (N*K bytes, read once) is the whole cost, so the kernel
 // is built like a plain streaming read: one CTA per SM owns a contiguous
-// range of 8-row units (balanced to within 8 rows) and warp 16 streams it
-// with TMA into a ring of 16 KB slots, each one 16-row tile x 1 KB of K
-// (64-byte swizzle, so a warp's 16-byte reads hit distinct banks).  Warps
+// range of 16-row tiles (balanced to within one tile) and warp 16 streams it
+// with TMA into a ring of 16 KB slots, each one tile x 1 KB of K (one box;
+// 64-byte swizzle, so a warp's 16-byte reads hit distinct banks).  Splitting
+// finer, into 8- or 4-row boxes, balances the SMs better but streams slower
+// on this part, and loses more than it gains.  Warps
 // 0..15 split every slot's K: warp w takes the 64-byte chunk w, and lane
 // (g, t) bytes [16t, 16t+16) of rows g and g+8.
 //
@@ -27,7 +29,7 @@
 // multiplied by 2^-s_m on the way out, exactly.  So every product of an
 // activation within that range is exact in FP32, as with BF16 operands.  The
 // row maxima are found at the start by all consumer warps together, while
-// the first weight copies are in flight.
+// the first weight copies and activation fragments are in flight.
 //
 // The activation fragments (L2-resident) come straight from global memory
 // into registers one K stage ahead of their use, are converted once per
@@ -195,10 +197,9 @@ __device__ __forceinline__ void consumers_sync() {
 // ---------------------------------------------------------------------------
 //   tmW   weights, wide (K % 64 == 0): 3-D (64 B, N rows, K/64 chunks), box
 //         (64, 16, 16): one slot; narrow: 2-D (K, N), box (64, 16): one chunk
-//   tmW8  the same with 8-row boxes (the last tile of an odd unit count)
 template <int MT, bool BS>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_fp8_gemv(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW8, int wide,
+    k_fp8_gemv(const __grid_constant__ CUtensorMap tmW, int wide,
                const uint16_t *__restrict__ X, const float *__restrict__ scale, uint16_t *__restrict__ out, int M,
                int N, int K) {
     constexpr int TG = group_tiles<MT>(), NS = slots<MT>();
@@ -209,14 +210,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     Bars *S = reinterpret_cast<Bars *>(red + red_floats<MT>());
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // this CTA's rows: a range of 8-row units, taken as 16-row tiles, the
-    // last one 8 rows when the unit count is odd
-    const int units = (N + 7) >> 3;
-    const int u_begin = (int)((int64_t)units * blockIdx.x / gridDim.x);
-    const int u_end = (int)((int64_t)units * (blockIdx.x + 1) / gridDim.x);
-    const int row_begin = 8 * u_begin, row_end = min(8 * u_end, N);
-    const int t_end = (u_end - u_begin + 1) >> 1;
-    const bool half_last = ((u_end - u_begin) & 1) != 0;
+    // this CTA's rows: a range of 16-row tiles (rows past N read as zeros)
+    const int tiles = (N + 15) >> 4;
+    const int t_begin = (int)((int64_t)tiles * blockIdx.x / gridDim.x);
+    const int t_end = (int)((int64_t)tiles * (blockIdx.x + 1) / gridDim.x) - t_begin;
+    const int row_begin = 16 * t_begin, row_end = min(16 * (t_begin + t_end), N);
     const int nst = (K + KS - 1) / KS;  // K stages
 
     if (threadIdx.x == 0) {
@@ -235,7 +233,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------- TMA producer
         if (lane == 0) {
             prefetch_tensormap(&tmW);
-            prefetch_tensormap(&tmW8);
             uint32_t it = 0;
             bool ok = true;
             for (int g0 = 0; g0 < t_end && ok; g0 += TG) {
@@ -248,18 +245,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
-                        const int tile = g0 + u;
-                        const bool h8 = half_last && tile == t_end - 1;
-                        const int rows = h8 ? 8 : 16;
-                        const CUtensorMap *map = h8 ? &tmW8 : &tmW;
                         uint8_t *dst = base + (size_t)s * SLOT;
-                        const int row0 = row_begin + 16 * tile;
-                        mbar_arrive_expect_tx(&S->full[s], (uint32_t)(nch * rows * CH));
+                        const int row0 = row_begin + 16 * (g0 + u);
+                        mbar_arrive_expect_tx(&S->full[s], (uint32_t)(nch * 16 * CH));
                         if (wide) {
-                            tma_load_3d(dst, map, &S->full[s], 0, row0, q * 16);
+                            tma_load_3d(dst, &tmW, &S->full[s], 0, row0, q * 16);
                         } else {
                             for (int c = 0; c < nch; c++)
-                                tma_load_2d(dst + c * rows * CH, map, &S->full[s], q * KS + c * CH, row0);
+                                tma_load_2d(dst + c * 16 * CH, &tmW, &S->full[s], q * KS + c * CH, row0);
                         }
                     }
                 }
@@ -281,38 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sbase = smem_u32(base);
 
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    // ---- each activation row's largest magnitude, found by all consumer
-    // warps together: warp w scans part w / M of row w % M (16 / M parts per
-    // row), up to eight 16-byte loads in flight per lane; the shuffles come
-    // after the loop, so every lane of the warp reaches them
-    {
-        const int parts = kConsumers / M, m = warp % M, p = warp / M;
-        uint32_t mx = 0;
-        if (p < parts) {
-            const int units = K >> 3;  // 16-byte units of a row
-            const int per = (units + parts - 1) / parts;
-            const int u0 = p * per, u1 = min(units, u0 + per);
-            const uint4 *xr = reinterpret_cast<const uint4 *>(X + (int64_t)m * K);
-            for (int u = u0 + lane; u < u1; u += 32 * 8) {
-                uint4 v[8];
-#pragma unroll
-                for (int j = 0; j < 8; j++) v[j] = u + 32 * j < u1 ? ldg_nc_v4(xr + u + 32 * j) : z;
-#pragma unroll
-                for (int j = 0; j < 8; j++)
-                    mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v[j].x & 0x7FFF7FFFu, v[j].y & 0x7FFF7FFFu),
-                                               __vmaxu2(v[j].z & 0x7FFF7FFFu, v[j].w & 0x7FFF7FFFu)));
-            }
-        }
-        mx = max(mx & 0xFFFFu, mx >> 16);
-        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-        if (lane == 0 && p < parts) atomicMax(&S->rowmax[m], mx);
-    }
-    consumers_sync();
-    const float xs0 = pow2i(row_shift(S->rowmax[g < M ? g : 0]));
-    const float xs1 = pow2i(row_shift(S->rowmax[(MT == 2 && g + 8 < M) ? g + 8 : 0]));
-
     // this lane's activation rows (g and, for MT == 2, g + 8) at K offset
-    // 64 * warp + 16 * t of every stage; rows past M read row 0 and are zeroed
+    // 64 * warp + 16 * t of every stage; rows past M read row 0 and are
+    // zeroed.  The first stage's fragments are requested before the row
+    // maxima below, so the two round trips overlap.
     const bool xv0 = g < M, xv1 = MT == 2 && g + 8 < M;
     const uint16_t *x0 = X + (int64_t)(xv0 ? g : 0) * K + CH * warp + 16 * t;
     const uint16_t *x1 = X + (int64_t)(xv1 ? g + 8 : 0) * K + CH * warp + 16 * t;
@@ -327,6 +292,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     uint4 nxa[2], nxb[2];
     load_x(0, nxa, nxb);
+
+    // ---- each activation row's largest magnitude, found by all consumer
+    // warps together: warp w scans part w / M of row w % M (16 / M parts per
+    // row), up to twelve 16-byte loads in flight per lane (a 5120-wide row
+    // of sixteen takes two round trips); the shuffles come after the loop,
+    // so every lane of the warp reaches them
+    {
+        constexpr int B = 12;
+        const int parts = kConsumers / M, m = warp % M, p = warp / M;
+        uint32_t mx = 0;
+        if (p < parts) {
+            const int units = K >> 3;  // 16-byte units of a row
+            const int per = (units + parts - 1) / parts;
+            const int u0 = p * per, u1 = min(units, u0 + per);
+            const uint4 *xr = reinterpret_cast<const uint4 *>(X + (int64_t)m * K);
+            for (int u = u0 + lane; u < u1; u += 32 * B) {
+                uint4 v[B];
+#pragma unroll
+                for (int j = 0; j < B; j++) v[j] = u + 32 * j < u1 ? ldg_nc_v4(xr + u + 32 * j) : z;
+#pragma unroll
+                for (int j = 0; j < B; j++)
+                    mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v[j].x & 0x7FFF7FFFu, v[j].y & 0x7FFF7FFFu),
+                                               __vmaxu2(v[j].z & 0x7FFF7FFFu, v[j].w & 0x7FFF7FFFu)));
+            }
+        }
+        mx = max(mx & 0xFFFFu, mx >> 16);
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (lane == 0 && p < parts) atomicMax(&S->rowmax[m], mx);
+    }
+    consumers_sync();
+    const float xs0 = pow2i(row_shift(S->rowmax[g < M ? g : 0]));
+    const float xs1 = pow2i(row_shift(S->rowmax[(MT == 2 && g + 8 < M) ? g + 8 : 0]));
 
     int s = 0;
     uint32_t ph = 0;
@@ -371,11 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok) ok = mbar_wait(&S->full[cs], cph, &g_timeouts);
                 ok = __all_sync(0xFFFFFFFFu, ok);
                 if (!ok) continue;
-                const bool h8 = half_last && g0 + u == t_end - 1;
                 if (active) {
-                    const uint32_t chunk = sbase + (uint32_t)cs * SLOT + warp * (h8 ? 8 : 16) * CH;
+                    const uint32_t chunk = sbase + (uint32_t)cs * SLOT + warp * 16 * CH;
                     f.wa = lds_v4(chunk + w_off(g, t));
-                    f.wb = h8 ? z : lds_v4(chunk + w_off(g + 8, t));
+                    f.wb = lds_v4(chunk + w_off(g + 8, t));
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S->empty[cs]);
@@ -427,22 +423,22 @@ static cudaError_t launch_mt(const uint16_t *in, const uint8_t *w, const float *
                                     (int)smem_bytes<MT>());
     });
     if (e != cudaSuccess) return e;
-    alignas(64) CUtensorMap tW, tW8;
+    alignas(64) CUtensorMap tW;
     const int wide = (k % CH) == 0;
     const uint64_t K = (uint64_t)k, N = (uint64_t)n;
     bool ok;
     if (wide) {
         const uint64_t d[3] = {CH, N, K / CH}, st[2] = {K, CH};
-        const uint32_t b16[3] = {CH, 16, 16}, b8[3] = {CH, 8, 16};
-        ok = make_tmap(&tW, w, 1, 3, d, st, b16, 64) && make_tmap(&tW8, w, 1, 3, d, st, b8, 64);
+        const uint32_t b16[3] = {CH, 16, 16};
+        ok = make_tmap(&tW, w, 1, 3, d, st, b16, 64);
     } else {
         const uint64_t d[2] = {K, N}, st[1] = {K};
-        const uint32_t b16[2] = {CH, 16}, b8[2] = {CH, 8};
-        ok = make_tmap(&tW, w, 1, 2, d, st, b16, 64) && make_tmap(&tW8, w, 1, 2, d, st, b8, 64);
+        const uint32_t b16[2] = {CH, 16};
+        ok = make_tmap(&tW, w, 1, 2, d, st, b16, 64);
     }
     if (!ok) return cudaErrorInvalidValue;
-    const int units = (n + 7) / 8;
-    const int grid = units < sm_count() ? units : sm_count();
+    const int tiles = (n + 15) / 16;
+    const int grid = tiles < sm_count() ? tiles : sm_count();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -453,7 +449,7 @@ static cudaError_t launch_mt(const uint16_t *in, const uint8_t *w, const float *
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_fp8_gemv<MT, BS>, tW, tW8, wide, in, scale, out, m, n, k);
+    return cudaLaunchKernelEx(&cfg, k_fp8_gemv<MT, BS>, tW, wide, in, scale, out, m, n, k);
 }
 
 template <bool BS>
