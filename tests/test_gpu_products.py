@@ -215,12 +215,11 @@ def test_gemv_cfg2(gemv_weight, m):
 
 
 def test_gemv_activation_range(gemv_weight):
-    """The GEMV runs its activations through FP16 with a power of two per row
-    and 64-element K chunk, so rows far from 1 in magnitude must still match
-    the oracle: a row scaled by 2^100, one by 2^-100, an all-zero row, and a
-    row whose largest element is 2^20 times its others; each row's result
-    must also equal the same row computed alone (a chunk's scale depends on
-    its own row only)."""
+    """The GEMV runs its activations through FP16 with a per-row power of two,
+    so rows far from 1 in magnitude must still match the oracle: a row
+    scaled by 2^100, one by 2^-100, an all-zero row, and a row whose largest
+    element is 2^20 times its others; each row's result must also equal the
+    same row computed alone (the scale is per row)."""
     wq, ws = gemv_weight
     base = synth.normal_bf16((4, 5120), 1.0, 2, 7)
     x = oracle.bf16_to_f32(base).astype(np.float32)
