@@ -400,9 +400,10 @@ def run_int8(a, w, sa, sw):
 
 
 # (128, 20224, 128) has 158 tiles: more than one per SM, so some CTAs take a
-# second tile
+# second tile; (2048, 1280, 256) has 160 (a short second round), and
+# (2000, 1280, 384) the same with a ragged last row tile.
 @pytest.mark.parametrize("mnk", [(64, 128, 128), (200, 300, 640), (129, 136, 1024), (1, 130, 256), (77, 131, 384),
-                                 (128, 20224, 128)])
+                                 (128, 20224, 128), (64, 128, 512), (2048, 1280, 256), (2000, 1280, 384)])
 def test_int8_small_and_ragged(mnk):
     m, n, k = mnk
     a_bf, w_bf = synth.w4a8_inputs(m, n, k, seed=1)
