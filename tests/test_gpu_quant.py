@@ -324,3 +324,37 @@ def test_quant_nvfp4_divisor_classes(scale2):
     op, os_ = oracle.quant_nvfp4(x, scale2)
     assert np.array_equal(gs, os_), f"scales differ at {np.argwhere(gs != os_)[:4]}"
     assert np.array_equal(gp, op), f"codes differ at {np.argwhere(gp != op)[:4]}"
+
+
+def test_quant_nvfp4_every_scale_at_every_boundary():
+    """Every finite positive E4M3 block scale, forced by a block whose
+    largest element is exactly 6 times its value (activation path, scale2 =
+    1), with the other fifteen elements on E2M1 code boundaries (exact ties),
+    on code values, and one BF16 step either side of a boundary, both signs:
+    the kernels' division-free code rule must give the oracle's codes bit for
+    bit for every divisor it meets."""
+    mags = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0]
+    rows = []
+    for code in range(1, 127):
+        v = np.float32(oracle.e4m3_value(code))
+        base = [np.float32(6.0) * v] + [np.float32(b) * v for b in mags]
+        for sign in (1.0, -1.0):
+            for step in (0, 1, -1):
+                blk = np.array(base[:1] + base[1:], np.float32)
+                body = blk[1:] * np.float32(sign)
+                bits = synth.to_bf16_bits(body).astype(np.int32)
+                if step:
+                    # one BF16 step away from zero (+1) or towards it (-1)
+                    bits = bits + step
+                body = oracle.bf16_to_f32(bits.astype(np.uint16))
+                block = np.zeros(16, np.float32)
+                block[0] = blk[0]
+                block[1:1 + len(body)] = body
+                rows.append(block)
+    x = synth.to_bf16_bits(np.stack(rows).reshape(-1, 32))
+    # the forced block maxima are exact in BF16, so every block's scale is its code
+    gp, gs = gpu_nvfp4(x, 1.0)
+    op, os_ = oracle.quant_nvfp4(x, 1.0)
+    assert np.array_equal(gs, os_), f"scales differ at {np.argwhere(gs != os_)[:4]}"
+    assert np.array_equal(gp, op), f"codes differ at {np.argwhere(gp != op)[:4]}"
+    assert len(set(gs.ravel().tolist())) >= 126
