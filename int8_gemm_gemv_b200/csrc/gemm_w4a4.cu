@@ -11,16 +11,20 @@
 // fed from L2.
 //
 // Per CTA (512 threads):
-//   warp 0        TMA producer.  A and weight halves go into a 5-stage ring;
+//   warp 0        TMA producer of A and the weight halves: a 5-stage ring;
 //                 their arrival is counted on the even CTA's barrier (the
-//                 MMA issuer's).  The raw scale tiles (A: own 128 rows, W:
-//                 all 256 rows) arrive on a local barrier.
+//                 MMA issuer's).
+//   warp 2        TMA producer of the raw scale tiles (A: own 128 rows, W:
+//                 all 256 rows), into a ring of their own that refills as
+//                 soon as the writers have moved a slot into tensor memory,
+//                 so a stage's scales land well before its A and W tiles.
 //   warps 12..15  scale-factor writers: the scale tiles arrive row-major
 //                 ([rows, 16 bytes] per 256-wide K block); the MMA reads its
 //                 scales from tensor memory where, in every 32-lane group,
-//                 lane i of column j holds row 32j+i.  They write that layout
-//                 with tcgen05.st (off the tensor core's queue) and tell the
-//                 even CTA.
+//                 lane i of column j holds row 32j+i.  Once the stage's
+//                 tensor-memory slot is free they write that layout with
+//                 tcgen05.st (off the tensor core's queue) and tell the even
+//                 CTA.
 //   warp 1        tensor-memory allocation for the pair; in the even CTA,
 //                 lane 0 issues the pair MMAs and commits them to both CTAs.
 //   warps 4..11   epilogue: tensor memory -> registers -> scale -> BF16 ->
@@ -55,7 +59,8 @@ constexpr int A_BYTES = BM * BK_BYTES;   // 16 KB
 constexpr int B_BYTES = BNH * BK_BYTES;  // 16 KB
 constexpr int SFA_BYTES = BM * 16;       // 2 KB
 constexpr int SFB_BYTES = BN * 16;       // 4 KB (all 256 weight rows)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int AB_STAGE_BYTES = A_BYTES + B_BYTES;      // 32 KB
+constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;  // 6 KB
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0;               // 256 FP32 columns
 constexpr int SF_COL = 256;              // per stage: 16 (A) + 32 (W)
@@ -69,7 +74,7 @@ constexpr int OUT_BOX_BYTES = OUT_BOX_COLS * 2 * OUT_BOX_ROWS;  // 4 KB
 constexpr int OUT_WARP_BYTES = OUT_BOX_BYTES;
 constexpr int OUT_BYTES = kEpiWarps * OUT_WARP_BYTES;             // 32 KB
 
-static_assert(STAGE_BYTES % 1024 == 0, "stages must stay 1024-byte aligned");
+static_assert(AB_STAGE_BYTES % 1024 == 0 && SF_STAGE_BYTES % 128 == 0, "stage alignment");
 static_assert(SF_COL + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
 
 static __device__ unsigned int g_timeouts;
@@ -79,12 +84,13 @@ struct Smem {
     uint64_t sf_full[STAGES];  // local: raw scale tiles landed
     uint64_t sfready[STAGES];  // even CTA: both CTAs' scales are in tensor memory
     uint64_t empty[STAGES];    // local: the pair MMAs of this stage are done
+    uint64_t sf_empty[STAGES]; // local: the scale slot's tiles are in tensor memory
     uint64_t tfull, tempty, drain;
     uint32_t tmem_base;
     uint32_t abort;
 };
 
-constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + OUT_BYTES + sizeof(Smem);
+constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * (AB_STAGE_BYTES + SF_STAGE_BYTES) + OUT_BYTES + sizeof(Smem);
 
 __device__ __forceinline__ bool aborted(volatile Smem *s) { return s->abort != 0; }
 
@@ -95,12 +101,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float scale_ab, const float *__restrict__ scale_b_dev, int M, int N, int K) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *out_stage = base + (size_t)STAGES * STAGE_BYTES;
+    uint8_t *sf_base = base + (size_t)STAGES * AB_STAGE_BYTES;
+    uint8_t *out_stage = sf_base + (size_t)STAGES * SF_STAGE_BYTES;
     Smem *S = reinterpret_cast<Smem *>(out_stage + OUT_BYTES);
-    auto a_tile = [&](int s) { return base + (size_t)s * STAGE_BYTES; };
-    auto b_tile = [&](int s) { return base + (size_t)s * STAGE_BYTES + A_BYTES; };
-    auto sfa_tile = [&](int s) { return base + (size_t)s * STAGE_BYTES + A_BYTES + B_BYTES; };
-    auto sfb_tile = [&](int s) { return base + (size_t)s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES; };
+    auto a_tile = [&](int s) { return base + (size_t)s * AB_STAGE_BYTES; };
+    auto b_tile = [&](int s) { return base + (size_t)s * AB_STAGE_BYTES + A_BYTES; };
+    auto sfa_tile = [&](int s) { return sf_base + (size_t)s * SF_STAGE_BYTES; };
+    auto sfb_tile = [&](int s) { return sf_base + (size_t)s * SF_STAGE_BYTES + SFA_BYTES; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();  // 0: issues the pair MMAs
@@ -115,6 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&S->sf_full[s], 1);
             mbar_init(&S->sfready[s], 2 * kSfWarps);
             mbar_init(&S->empty[s], 1);
+            mbar_init(&S->sf_empty[s], kSfWarps);
         }
         mbar_init(&S->tfull, 1);
         mbar_init(&S->tempty, 2 * kEpiWarps);
@@ -135,12 +143,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto leader = [&](uint64_t *bar) { return mapa_shared(smem_u32(bar), 0); };
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------- TMA producer: A, W
         if (lane == 0) {
             prefetch_tensormap(&tmA);
             prefetch_tensormap(&tmB);
-            prefetch_tensormap(&tmSFA);
-            prefetch_tensormap(&tmSFB);
             // everything above overlapped the previous kernel of the stream
             // (programmatic stream serialization); global memory is read
             // from here on, after it has completed.  Every other role's
@@ -162,6 +168,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t abar = leader(&S->ab_full[s]);
                     tma_load_2d_pair(a_tile(s), &tmA, abar, kb * BK_BYTES, arow);
                     tma_load_2d_pair(b_tile(s), &tmB, abar, kb * BK_BYTES, brow);
+                }
+            }
+            if (!ok) S->abort = 1;
+        }
+    } else if (warp == 2) {
+        // -------------------------------------- TMA producer: scale tiles
+        // Its own ring: a slot is refilled as soon as the writers have moved
+        // its tiles into tensor memory, so the scales of a stage arrive
+        // several stages before its A and W tiles.
+        if (lane == 0) {
+            prefetch_tensormap(&tmSFA);
+            prefetch_tensormap(&tmSFB);
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += npairs) {
+                const int mt = t % tiles_m, nt = t / tiles_m;
+                const int arow = mt * 2 * BM + (int)rank * BM;
+                for (int kb = 0; kb < nkb; kb++, it++) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(&S->sf_empty[s], ph ^ 1, &g_timeouts) || aborted(S)) {
+                        ok = false;
+                        break;
+                    }
                     mbar_arrive_expect_tx(&S->sf_full[s], SFA_BYTES + SFB_BYTES);
                     tma_load_2d(sfa_tile(s), &tmSFA, &S->sf_full[s], kb * 16, arow);
                     tma_load_2d(sfb_tile(s), &tmSFB, &S->sf_full[s], kb * 16, nt * BN);
@@ -185,10 +216,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < nkb; kb++, it++) {
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
-                if (!mbar_wait(&S->sf_full[s], ph, &g_timeouts) || aborted(S)) {
+                // the stage's tiles, and its tensor-memory slot: free once the
+                // pair MMAs of the stage STAGES earlier are done
+                if (!mbar_wait(&S->sf_full[s], ph, &g_timeouts) || !mbar_wait(&S->empty[s], ph ^ 1, &g_timeouts) ||
+                    aborted(S)) {
                     ok = false;
                     break;
                 }
+                tc_fence_after();
                 // raw tile: row r at r*16 bytes, word j = the 4 scales of MMA step j
                 const uint4 *sa = reinterpret_cast<const uint4 *>(sfa_tile(s));
                 const uint4 *sb = reinterpret_cast<const uint4 *>(sfb_tile(s));
@@ -219,7 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(leader(&S->sfready[s]));
+                if (lane == 0) {
+                    mbar_arrive(&S->sf_empty[s]);
+                    mbar_arrive_cluster(leader(&S->sfready[s]));
+                }
             }
         }
         if (!ok && lane == 0) S->abort = 1;
