@@ -65,7 +65,7 @@ __host__ __device__ constexpr int act_box_rows(int m) {
 }
 
 struct Smem {
-    uint64_t full[8], sfready[8], empty[8];
+    uint64_t full[8], sf_full[8], sfready[8], empty[8];
     uint64_t tfull, tempty, drain;
     uint32_t tmem_base;
     uint32_t abort;
@@ -125,11 +125,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
     }
-    const uint32_t data_bytes = W_BYTES + SFW_BYTES + (uint32_t)ma * (BK_BYTES + 16);
+    // per stage: the scale tiles on their own barrier, requested first, so the
+    // writers move them into tensor memory while the operand tiles land
+    const uint32_t sf_bytes = SFW_BYTES + (uint32_t)ma * 16, ab_bytes = W_BYTES + (uint32_t)ma * BK_BYTES;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
             mbar_init(&S->full[s], 1);
+            mbar_init(&S->sf_full[s], 1);
             mbar_init(&S->sfready[s], 4);
             mbar_init(&S->empty[s], 1);
         }
@@ -168,18 +171,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&S->full[s], data_bytes);
+                    mbar_arrive_expect_tx(&S->sf_full[s], sf_bytes);
+                    tma_load_2d(sfw_tile(s), &tmSFW, &S->sf_full[s], kb * 16, t * BW);
+                    tma_load_2d(sfa_tile(s), &tmSFA, &S->sf_full[s], kb * 16, 0);
+                    mbar_arrive_expect_tx(&S->full[s], ab_bytes);
                     tma_load_2d(w_tile(s), &tmW, &S->full[s], kb * BK_BYTES, t * BW);
                     tma_load_2d(a_tile(s), &tmA, &S->full[s], kb * BK_BYTES, 0);
-                    tma_load_2d(sfw_tile(s), &tmSFW, &S->full[s], kb * 16, t * BW);
-                    tma_load_2d(sfa_tile(s), &tmSFA, &S->full[s], kb * 16, 0);
                 }
             }
             if (!ok) {
                 S->abort = 1;
                 // let the copies already issued land before the CTA can exit
                 const uint32_t first = it > STAGES ? it - STAGES : 0;
-                for (uint32_t i = first; i < it; i++) mbar_wait(&S->full[i % STAGES], (i / STAGES) & 1, &g_timeouts);
+                for (uint32_t i = first; i < it; i++) {
+                    mbar_wait(&S->sf_full[i % STAGES], (i / STAGES) & 1, &g_timeouts);
+                    mbar_wait(&S->full[i % STAGES], (i / STAGES) & 1, &g_timeouts);
+                }
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -191,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             for (int kb = 0; kb < nkb; kb++, it++) {
                 const int s = it % STAGES;
-                if (!mbar_wait(&S->full[s], (it / STAGES) & 1, &g_timeouts) || aborted(S)) {
+                if (!mbar_wait(&S->sf_full[s], (it / STAGES) & 1, &g_timeouts) || aborted(S)) {
                     ok = false;
                     break;
                 }
