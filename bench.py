@@ -584,7 +584,12 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
     bsq.quant_act_int8_per32(a_list[0], ai, ais, m, k, stream)
     del a_list
     out = torch.empty((m, n), dtype=torch.int16, device=dev)
-    t = time_launches(torch, stream, lambda: bsq.int8_blockscaled_gemm(ai, wi, ais, wis, out, m, n, k, stream), 5)
+    t_plain = time_launches(torch, stream, lambda: bsq.int8_blockscaled_gemm(ai, wi, ais, wis, out, m, n, k, stream), 5)
+    # the workspace form: the partial last round of tiles split along K
+    ws_bytes = bsq.int8_gemm_workspace_bytes()
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    t = time_launches(torch, stream,
+                      lambda: bsq.int8_blockscaled_gemm_ws(ai, wi, ais, wis, out, ws, ws_bytes, m, n, k, stream), 5)
     tops = 2.0 * m * n * k / t / 1e12
     # The fold's own roofline: two FP32 lane operations (the scale product and
     # the FMA) per output and 32-block, against every SM's 128 FP32 lanes at
@@ -595,7 +600,9 @@ def measure_rows(torch, bsq, dev, stream, peaks, peak_src):
     rows[f"a7_int8_blockscaled_gemm_{m}x{n}x{k}"] = {
         "us": round(t * 1e6, 1), "tops": round(tops, 1), "frac_int8": round(tops / (bf16 * RATIO_INT8), 4),
         "fold_gops": round(fold_rate / 1e9, 1), "fold_peak_gops": round(fold_peak / 1e9, 1),
-        "frac_fold": round(fold_rate / fold_peak, 4), "bound": "alu (per-32 FP32 fold on CUDA cores)"}
+        "frac_fold": round(fold_rate / fold_peak, 4), "bound": "alu (per-32 FP32 fold on CUDA cores)",
+        "call": "int8_blockscaled_gemm_ws (workspace split of the last round)",
+        "us_without_workspace": round(t_plain * 1e6, 1)}
     return rows
 
 

@@ -266,6 +266,33 @@ BSQ_API bsq_status int8_blockscaled_gemm(const int8_t *a_i8, const int8_t *w_i8,
                                  bsq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * int8_blockscaled_gemm_ws -- int8_blockscaled_gemm with a caller workspace,
+ * in the caller-owned-scratch style of gemm_dense_int8.rs
+ * `int8_gemm_faith2_prefill`.  Tiles of 128 x 128 outputs go round-robin over
+ * one CTA per SM; when the last round would leave most SMs idle, each of its
+ * tiles is split along K into up to four pieces on otherwise idle SMs, and
+ * the pieces' FP32 sums are added through the workspace in piece order.
+ *   workspace  device memory of int8_gemm_workspace_bytes() bytes, 16-byte
+ *              aligned, zeroed once before its first use (every call leaves
+ *              its counters at zero again).  Calls that share a workspace
+ *              must not overlap on the GPU; stream-ordered calls may share.
+ *   ws_bytes   its size.
+ * Same result definition and tolerance as int8_blockscaled_gemm; the outputs
+ * of a split tile are summed piece by piece, so they may differ from that
+ * call in the last bits, but never from run to run.
+ * Errors: those of int8_blockscaled_gemm; workspace NULL or ws_bytes too
+ * small -> INVALID_ARG; misaligned -> MISALIGNED.
+ * ---------------------------------------------------------------------- */
+BSQ_API bsq_status int8_blockscaled_gemm_ws(const int8_t *a_i8, const int8_t *w_i8,
+                                    const float *a_scale, const float *w_scale,
+                                    uint16_t *out, void *workspace, size_t ws_bytes,
+                                    int m, int n, int k, bsq_stream_t stream);
+
+/* Workspace bytes int8_blockscaled_gemm_ws needs on the current device (64 KB
+ * and 4 bytes per SM, for any shape); 0 if the device cannot be queried. */
+BSQ_API size_t int8_gemm_workspace_bytes(void);
+
+/* ------------------------------------------------------------------------
  * int8_w4a8_prefill -- gemm_dense_int8.rs, `int8_gemm_faith2_prefill`:
  * quant_act_int8_per32 into the caller's scratch, then
  * int8_blockscaled_gemm, two launches on `stream`.

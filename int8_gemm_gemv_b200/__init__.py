@@ -58,6 +58,7 @@ _SIGS = {
     "requant_w_nvfp4_int8": [_P, _P, _F, _P, _P, _I, _I, _P],
     "quant_act_int8_per32": [_P, _P, _P, _I, _I, _P],
     "int8_blockscaled_gemm": [_P, _P, _P, _P, _P, _I, _I, _I, _P],
+    "int8_blockscaled_gemm_ws": [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _P],
     "int8_w4a8_prefill": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P],
     "int8_w4a8_prefill_noalloc": [_P, _P, _P, _P, _I, _I, _I, _P],
     "requant_blockfp8_to_rowwise": [_I, _P, _P, _I, _I, _P, _P, ctypes.POINTER(_P), ctypes.POINTER(_P), _P],
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.bsq_debug_take_cuda_error.restype = ctypes.c_int
         L.bsq_debug_cuda_error_string.argtypes = [ctypes.c_int]
         L.bsq_debug_cuda_error_string.restype = ctypes.c_char_p
+        L.int8_gemm_workspace_bytes.argtypes = []
+        L.int8_gemm_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -186,6 +189,19 @@ def quant_act_int8_per32(a, a_i8, a_scale, m, k, stream=None):
 def int8_blockscaled_gemm(a_i8, w_i8, a_scale, w_scale, out, m, n, k, stream=None):
     _call("int8_blockscaled_gemm", _ptr(a_i8), _ptr(w_i8), _ptr(a_scale), _ptr(w_scale), _ptr(out), m, n, k,
           _stream(stream))
+
+
+def int8_gemm_workspace_bytes():
+    """Bytes of the workspace int8_blockscaled_gemm_ws needs on the current
+    device (0 when it cannot be queried)."""
+    return int(lib().int8_gemm_workspace_bytes())
+
+
+def int8_blockscaled_gemm_ws(a_i8, w_i8, a_scale, w_scale, out, workspace, ws_bytes, m, n, k, stream=None):
+    """int8_blockscaled_gemm with a workspace (zeroed once before first use)
+    that lets a partial last round of tiles be split along K."""
+    _call("int8_blockscaled_gemm_ws", _ptr(a_i8), _ptr(w_i8), _ptr(a_scale), _ptr(w_scale), _ptr(out),
+          _ptr(workspace), ws_bytes, m, n, k, _stream(stream))
 
 
 def int8_w4a8_prefill(a_bf16, w_i8, w_scale, a_i8_scratch, a_scale_scratch, out, m, n, k, stream=None):

@@ -170,6 +170,27 @@ bsq_status int8_blockscaled_gemm(const int8_t *a_i8, const int8_t *w_i8, const f
     return cuda_status(bsq::launch_int8_blockscaled_gemm(a_i8, w_i8, a_scale, w_scale, out, m, n, k, cs(stream)));
 }
 
+size_t int8_gemm_workspace_bytes(void) {
+    // ensure a context on the caller's current device, as the launchers do
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    return bsq::int8_gemm_workspace_bytes();
+}
+
+bsq_status int8_blockscaled_gemm_ws(const int8_t *a_i8, const int8_t *w_i8, const float *a_scale,
+                                    const float *w_scale, uint16_t *out, void *workspace, size_t ws_bytes, int m,
+                                    int n, int k, bsq_stream_t stream) {
+    bsq_status st = check_int8_gemm(a_i8, w_i8, a_scale, w_scale, out, m, n, k);
+    if (st != BSQ_OK || m == 0 || n == 0) return st;
+    if (!workspace) return BSQ_ERR_INVALID_ARG;
+    if (!al16(workspace)) return BSQ_ERR_MISALIGNED;
+    const size_t need = bsq::int8_gemm_workspace_bytes();
+    if (need == 0) return BSQ_ERR_CUDA;
+    if (ws_bytes < need) return BSQ_ERR_INVALID_ARG;
+    return cuda_status(
+        bsq::launch_int8_blockscaled_gemm_ws(a_i8, w_i8, a_scale, w_scale, out, workspace, m, n, k, cs(stream)));
+}
+
 bsq_status int8_w4a8_prefill(const uint16_t *a_bf16, const int8_t *w_i8, const float *w_scale,
                              int8_t *a_i8_scratch, float *a_scale_scratch, uint16_t *out, int m, int n, int k,
                              bsq_stream_t stream) {

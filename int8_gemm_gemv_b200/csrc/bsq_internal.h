@@ -98,6 +98,13 @@ cudaError_t launch_fp8_gemm_rowscale(const uint8_t *a, const float *a_scale, con
 cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const float *a_scale,
                                          const float *w_scale, uint16_t *out, int m, int n, int k,
                                          cudaStream_t s);
+// The same with a workspace of int8_gemm_workspace_bytes() bytes (zeroed once
+// before first use; calls sharing it must be stream-ordered): a last round of
+// tiles that would leave SMs idle is split along K (gemm_int8.cu).
+cudaError_t launch_int8_blockscaled_gemm_ws(const int8_t *a, const int8_t *w, const float *a_scale,
+                                            const float *w_scale, uint16_t *out, void *workspace, int m, int n,
+                                            int k, cudaStream_t s);
+size_t int8_gemm_workspace_bytes();
 
 // ---- tensor maps (tma.cu) ----
 // 2-D row-major tensor of `rows` x `cols` elements of `elem_bytes` bytes,

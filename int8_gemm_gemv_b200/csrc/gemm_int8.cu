@@ -25,6 +25,13 @@
 // each half is folded while the next is in flight.  Four fold warps per
 // SM sub-partition hide the remaining latency; to fit them, warps 0-3 give
 // up registers (setmaxnreg).
+//
+// Tiles go round-robin over one CTA per SM.  With a caller workspace, a last
+// round that would leave most SMs idle is split along K: each of its tiles
+// becomes S pieces on S CTAs.  A piece stores its FP32 sums in the
+// workspace and counts itself in the tile's counter; the piece that counts
+// last adds all S in piece order (so the result never depends on which
+// finished last), stores the tile and puts the counter back to zero.
 #include "bsq_common.cuh"
 
 namespace bsq {
@@ -56,6 +63,8 @@ struct Smem {
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
+    uint32_t last_piece;  // this CTA's piece was the last of its tile
+    uint64_t fold_bar;    // the 16 fold warps of a split-tile hand-off (two phases)
 };
 
 constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Smem);
@@ -85,10 +94,47 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     return d;
 }
 
+// The i-th tile of this CTA: tile t over K blocks [kb0, kb1) (blocks of BK),
+// piece `piece` of `split` pieces when split > 1.  False past the CTA's last
+// tile.  Every role walks the same list.
+struct ITile {
+    int t, kb0, kb1, piece;
+};
+__device__ __forceinline__ bool int8_tile(int i, int num_tiles, int nkb, int split, ITile &o) {
+    const int G = gridDim.x, b = blockIdx.x;
+    const int full = num_tiles / G, rem = num_tiles % G;
+    if (i < full) {
+        o = {b + i * G, 0, nkb, 0};
+        return true;
+    }
+    if (i != full || rem == 0) return false;
+    if (split > 1) {
+        if (b >= rem * split) return false;
+        const int r = b / split, p = b % split;
+        o = {full * G + r, p * nkb / split, (p + 1) * nkb / split, p};
+        return true;
+    }
+    if (b >= rem) return false;
+    o = {full * G + b, 0, nkb, 0};
+    return true;
+}
+
+// Pieces per tile of the last round: up to four, as many as the idle CTAs
+// allow, 1 when that round is full or K has a single block.
+__host__ __device__ __forceinline__ int int8_split(int num_tiles, int grid, int nkb) {
+    const int rem = num_tiles % grid;
+    if (rem == 0) return 1;
+    int sp = grid / rem;
+    sp = sp < 4 ? sp : 4;
+    sp = sp < nkb ? sp : nkb;
+    return sp > 1 ? sp : 1;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_int8_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSW,
-                uint16_t *__restrict__ out, int M, int N, int K) {
+                uint16_t *__restrict__ out, int M, int N, int K, float *__restrict__ ws_part,
+                uint32_t *__restrict__ ws_cnt, int split) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Smem *S = reinterpret_cast<Smem *>(base + (size_t)STAGES * STAGE_BYTES);
@@ -115,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&S->acc_empty[b], NFOLD);
         }
         mbar_init(&S->drain, 1);
+        mbar_init(&S->fold_bar, NFOLD);
         S->abort = 0;
         fence_mbar_init();
     }
@@ -136,9 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tensormap(&tmSW);
             uint32_t it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                const int mt = t % tiles_m, nt = t / tiles_m;
-                for (int kb = 0; kb < nkb; kb++, it++) {
+            ITile tl;
+            for (int ti = 0; ok && int8_tile(ti, num_tiles, nkb, split, tl); ti++) {
+                const int mt = tl.t % tiles_m, nt = tl.t / tiles_m;
+                for (int kb = tl.kb0; kb < tl.kb1; kb++, it++) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!mbar_wait(&S->empty[s], ph ^ 1, &g_timeouts) || aborted(S)) {
@@ -162,8 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // W scales: [n][4] -> [4][n], in place
         uint32_t it = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-            for (int kb = 0; kb < nkb; kb++, it++) {
+        ITile tl;
+        for (int ti = 0; ok && int8_tile(ti, num_tiles, nkb, split, tl); ti++) {
+            for (int kb = tl.kb0; kb < tl.kb1; kb++, it++) {
                 const int s = it % STAGES;
                 if (!mbar_wait(&S->full[s], (it / STAGES) & 1, &g_timeouts) || aborted(S)) {
                     ok = false;
@@ -191,8 +240,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idesc = idesc_s8(BM, BN);
             uint32_t it = 0, gs = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                for (int kb = 0; kb < nkb && ok; kb++, it++) {
+            ITile tl;
+            for (int ti = 0; ok && int8_tile(ti, num_tiles, nkb, split, tl); ti++) {
+                for (int kb = tl.kb0; kb < tl.kb1 && ok; kb++, it++) {
                     const int s = it % STAGES;
                     if (!mbar_wait(&S->full[s], (it / STAGES) & 1, &g_timeouts) || aborted(S)) {
                         ok = false;
@@ -244,8 +294,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fma2(make_float2((float)(int)R[4 * g + 2], (float)(int)R[4 * g + 3]), c1v, acc[4 * u0 + 4 + g]);
             }
         };
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-            const int mt = t % tiles_m, nt = t / tiles_m;
+        auto store_tile = [&](int mt, int nt) {
+            // rows r0 + 8u, column pairs c0 + 8g
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int row = mt * BM + r0 + 8 * u;
+                if (row >= M) continue;
+                uint16_t *orow = out + (int64_t)row * N;
+#pragma unroll
+                for (int g = 0; g < 4; g++) {
+                    const int col = nt * BN + c0 + 8 * g;
+                    const float2 v = acc[4 * u + g];
+                    if ((N & 1) == 0 && col + 1 < N) {
+                        *reinterpret_cast<uint32_t *>(orow + col) = pack_bf16x2(v.x, v.y);
+                    } else {
+                        if (col < N) orow[col] = __bfloat16_as_ushort(__float2bfloat16_rn(v.x));
+                        if (col + 1 < N) orow[col + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(v.y));
+                    }
+                }
+            }
+        };
+        ITile tl;
+        for (int ti = 0; ok && int8_tile(ti, num_tiles, nkb, split, tl); ti++) {
+            const int mt = tl.t % tiles_m, nt = tl.t / tiles_m;
 #pragma unroll
             for (int i = 0; i < 16; i++) acc[i] = make_float2(0.0f, 0.0f);
             if (!wait_full(gs)) {
@@ -254,14 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_ld_16x256b_x4(tq + (gs % NACC) * BN, RA);
             tmem_ld_wait();
-            for (int kb = 0; kb < nkb && ok; kb++, it++) {
+            for (int kb = tl.kb0; kb < tl.kb1 && ok; kb++, it++) {
                 const int s = it % STAGES;
                 if (!mbar_wait(&S->swready[s], (it / STAGES) & 1, &g_timeouts) || aborted(S)) {
                     ok = false;
                     break;
                 }
                 const float *sat = sa_tile(s);
-                const bool last = kb == nkb - 1;
+                const bool last = kb == tl.kb1 - 1;
 #pragma unroll
                 for (int j = 0; j < 4; j++, gs++) {
                     // Upper half of block gs is in RA.  Load the lower half,
@@ -301,24 +372,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) S->abort = 1;
                 break;
             }
-            // epilogue: rows r0 + 8u, column pairs c0 + 8g
+            const int tail0 = num_tiles - num_tiles % (int)gridDim.x;  // first tile of the last round
+            if (split > 1 && tl.t >= tail0) {
+                // a piece of a split tile (the CTA's last tile): FP32 sums to
+                // the workspace, 128 bytes per fold thread; the last piece to
+                // count adds them.  The fold warps meet on an mbarrier with
+                // the usual bounded waits (a warp that timed out earlier never
+                // arrives, and the others give up after the limit).
+                const int ft = threadIdx.x - 4 * 32;  // 0 .. 511
+                const int r = tl.t - tail0;
+                float4 *mine = reinterpret_cast<float4 *>(ws_part + ((size_t)(r * split + tl.piece) * 512 + ft) * 32);
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int row = mt * BM + r0 + 8 * u;
-                if (row >= M) continue;
-                uint16_t *orow = out + (int64_t)row * N;
-#pragma unroll
-                for (int g = 0; g < 4; g++) {
-                    const int col = nt * BN + c0 + 8 * g;
-                    const float2 v = acc[4 * u + g];
-                    if ((N & 1) == 0 && col + 1 < N) {
-                        *reinterpret_cast<uint32_t *>(orow + col) = pack_bf16x2(v.x, v.y);
-                    } else {
-                        if (col < N) orow[col] = __bfloat16_as_ushort(__float2bfloat16_rn(v.x));
-                        if (col + 1 < N) orow[col + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(v.y));
-                    }
+                for (int i = 0; i < 8; i++)
+                    mine[i] = make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x, acc[2 * i + 1].y);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S->fold_bar);
+                if (!mbar_wait(&S->fold_bar, 0, &g_timeouts)) {  // every fold thread's sums are stored
+                    if (lane == 0) S->abort = 1;
+                    break;
                 }
+                if (ft == 0) {
+                    __threadfence();
+                    S->last_piece = atomicAdd(&ws_cnt[r], 1u) == (uint32_t)(split - 1);
+                    __threadfence();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S->fold_bar);
+                if (!mbar_wait(&S->fold_bar, 1, &g_timeouts)) {
+                    if (lane == 0) S->abort = 1;
+                    break;
+                }
+                if (S->last_piece) {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) acc[i] = make_float2(0.0f, 0.0f);
+                    for (int p = 0; p < split; p++) {  // piece order, whichever came last
+                        const float4 *src =
+                            reinterpret_cast<const float4 *>(ws_part + ((size_t)(r * split + p) * 512 + ft) * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; i++) {
+                            const float4 v = __ldcg(src + i);
+                            acc[2 * i].x += v.x;
+                            acc[2 * i].y += v.y;
+                            acc[2 * i + 1].x += v.z;
+                            acc[2 * i + 1].y += v.w;
+                        }
+                    }
+                    store_tile(mt, nt);
+                    if (ft == 0) ws_cnt[r] = 0;  // ready for the next call on this workspace
+                }
+                continue;
             }
+            store_tile(mt, nt);
         }
     }
 
@@ -339,9 +443,16 @@ uint32_t take_timeouts_gemm_int8() {
     return v;
 }
 
-cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const float *a_scale,
-                                         const float *w_scale, uint16_t *out, int m, int n, int k,
-                                         cudaStream_t s) {
+// Workspace of the tail split: one 64 KB piece of FP32 sums and one
+// counter per SM (a split never has more pieces or tiles than CTAs).
+static size_t ws_part_bytes() { return (size_t)sm_count() * 512 * 32 * 4; }
+size_t int8_gemm_workspace_bytes() {
+    const int sms = sm_count();
+    return sms > 0 ? ws_part_bytes() + (size_t)sms * 4 : 0;
+}
+
+static cudaError_t launch_int8(const int8_t *a, const int8_t *w, const float *a_scale, const float *w_scale,
+                               uint16_t *out, void *ws, int m, int n, int k, cudaStream_t s) {
     alignas(64) CUtensorMap tA, tB, tSA, tSW;
     const uint64_t kblk = (uint64_t)k / 32;
     if (!make_tmap_2d(&tA, a, 1, k, m, k, BK, BM, true, false) ||
@@ -362,9 +473,24 @@ cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const
     if (e != cudaSuccess) return e;
     const int tiles = ((m + BM - 1) / BM) * ((n + BN - 1) / BN);
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    k_int8_gemm<<<grid, kThreads, kSmemBytes, s>>>(tA, tB, tSA, tSW, out, m, n, k);
+    const int split = ws ? int8_split(tiles, grid, k / BK) : 1;
+    float *ws_part = ws ? static_cast<float *>(ws) : nullptr;
+    uint32_t *ws_cnt = ws ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + ws_part_bytes()) : nullptr;
+    k_int8_gemm<<<grid, kThreads, kSmemBytes, s>>>(tA, tB, tSA, tSW, out, m, n, k, ws_part, ws_cnt, split);
     note_launch();
     return cudaGetLastError();
+}
+
+cudaError_t launch_int8_blockscaled_gemm(const int8_t *a, const int8_t *w, const float *a_scale,
+                                         const float *w_scale, uint16_t *out, int m, int n, int k,
+                                         cudaStream_t s) {
+    return launch_int8(a, w, a_scale, w_scale, out, nullptr, m, n, k, s);
+}
+
+cudaError_t launch_int8_blockscaled_gemm_ws(const int8_t *a, const int8_t *w, const float *a_scale,
+                                            const float *w_scale, uint16_t *out, void *workspace, int m, int n,
+                                            int k, cudaStream_t s) {
+    return launch_int8(a, w, a_scale, w_scale, out, workspace, m, n, k, s);
 }
 
 }  // namespace bsq

@@ -4,7 +4,8 @@
 
 Inputs are random codes in device memory (the kernel's cost does not depend
 on their values beyond power); nothing is checked.  Kinds: w4a4 (M <= 128
-runs the few-row kernel), fp8gemm, int8gemm, gemv, gemv_bs (block-scaled),
+runs the few-row kernel), fp8gemm, int8gemm, int8gemm_ws (with the
+tail-splitting workspace), gemv, gemv_bs (block-scaled),
 quant_nvfp4, quant_rowfp8, quant_int8, requant_w, requant_block.
 """
 from __future__ import annotations
@@ -39,7 +40,7 @@ def main():
     def bf16(shape, std=1.0):
         return (torch.randn(shape, device=dev, generator=g) * std).to(torch.bfloat16)
 
-    out = torch.empty((m, n), dtype=torch.int16, device=dev) if a.kind in ("w4a4", "fp8gemm", "int8gemm", "gemv",
+    out = torch.empty((m, n), dtype=torch.int16, device=dev) if a.kind in ("w4a4", "fp8gemm", "int8gemm", "int8gemm_ws", "gemv",
                                                                           "gemv_bs") else None
     if a.kind == "w4a4":
         ap, asf, wp, wsf = u8((m, k // 2)), u8((m, k // 16), 0x30, 0x40), u8((n, k // 2)), u8((n, k // 16), 0x30, 0x40)
@@ -48,11 +49,16 @@ def main():
         x, w = u8((m, k), 0, 0x7F), u8((n, k), 0, 0x7F)
         sa, sw = torch.rand(m, device=dev), torch.rand(n, device=dev)
         fn = lambda: bsq.fp8_gemm_rowscale(x, sa, w, sw, out, m, n, k)
-    elif a.kind == "int8gemm":
+    elif a.kind in ("int8gemm", "int8gemm_ws"):
         x = torch.randint(-127, 128, (m, k), dtype=torch.int8, device=dev)
         w = torch.randint(-127, 128, (n, k), dtype=torch.int8, device=dev)
         sa, sw = torch.rand(m, k // 32, device=dev), torch.rand(n, k // 32, device=dev)
-        fn = lambda: bsq.int8_blockscaled_gemm(x, w, sa, sw, out, m, n, k)
+        if a.kind == "int8gemm":
+            fn = lambda: bsq.int8_blockscaled_gemm(x, w, sa, sw, out, m, n, k)
+        else:
+            nb = bsq.int8_gemm_workspace_bytes()
+            ws = torch.zeros(nb, dtype=torch.uint8, device=dev)
+            fn = lambda: bsq.int8_blockscaled_gemm_ws(x, w, sa, sw, out, ws, nb, m, n, k)
     elif a.kind == "gemv_bs":
         x, w = bf16((m, k)), u8((n, k), 0, 0x7F)
         S = torch.rand(n // 128, k // 128, device=dev)

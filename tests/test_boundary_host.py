@@ -150,3 +150,18 @@ def test_binding_rejects_host_tensors():
     torch = pytest.importorskip("torch")
     with pytest.raises(ValueError):
         bsq.quant_rowwise_fp8(torch.zeros(4, 16, dtype=torch.bfloat16), A16, A16b, 4, 16, stream=0)
+
+
+def test_int8_ws_validation():
+    L = bsq.lib()
+    n0 = bsq.debug_launch_count()
+    # NULL workspace, misaligned workspace; nothing launches
+    assert L.int8_blockscaled_gemm_ws(A16, A16b, A16c, A16d, A16e, None, 1 << 24, 128, 128, 128, None) == \
+        bsq.BSQ_ERR_INVALID_ARG
+    assert L.int8_blockscaled_gemm_ws(A16, A16b, A16c, A16d, A16e, A16 + 8, 1 << 24, 128, 128, 128, None) == \
+        bsq.BSQ_ERR_MISALIGNED
+    # the shape checks of the plain call come first
+    assert L.int8_blockscaled_gemm_ws(A16, A16b, A16c, A16d, A16e, A16, 1 << 24, 128, 128, 96, None) == \
+        bsq.BSQ_ERR_UNSUPPORTED
+    assert L.int8_blockscaled_gemm_ws(A16, A16b, A16c, A16d, A16e, A16, 1 << 24, 0, 128, 128, None) == bsq.BSQ_OK
+    assert bsq.debug_launch_count() == n0

@@ -73,6 +73,25 @@ def test_int8_full_k_bit_exact():
     _assert_bits(host(out, np.uint16)[rows], ob, "int8 2048x5120x17408 exact")
 
 
+@pytest.mark.gpu
+def test_int8_ws_full_k_bit_exact():
+    """The workspace form at the benchmark shape: 640 tiles on 148 SMs, so the
+    last 48 tiles (output columns 4736..5119) are split along K into three
+    pieces each.  Exact sums regardless of order, so bit-exact; every sampled
+    row crosses the split tiles."""
+    m, n, k = 2048, 5120, 17408
+    a, w, sa, sw = int8_sparse(m, n, k, seed=3)
+    out = bf16_out((m, n))
+    nbytes = bsq.int8_gemm_workspace_bytes()
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    bsq.int8_blockscaled_gemm_ws(to_dev(a), to_dev(w), to_dev(sa), to_dev(sw), out, ws, nbytes, m, n, k)
+    torch.cuda.synchronize()
+    assert bsq.debug_take_timeouts() == 0
+    rows = sample_rows(m, 10, 3)
+    ob, _, _ = oracle.int8_blockscaled_gemm(a, w, sa, sw, rows=rows)
+    _assert_bits(host(out, np.uint16)[rows], ob, "int8 ws 2048x5120x17408 exact")
+
+
 # --------------------------------------------- power of the design (CPU) ---
 
 def _changed_share(before, after):

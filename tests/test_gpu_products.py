@@ -416,6 +416,55 @@ def test_int8_small_and_ragged(mnk):
     check_tol(g, ob, ab, f"int8 {mnk}")
 
 
+def run_int8_ws(a, w, sa, sw, ws=None):
+    m, k = a.shape
+    n = w.shape[0]
+    out = bf16_out((m, n))
+    nbytes = bsq.int8_gemm_workspace_bytes()
+    if ws is None:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    bsq.int8_blockscaled_gemm_ws(to_dev(a), to_dev(w), to_dev(sa), to_dev(sw), out, ws, nbytes, m, n, k)
+    torch.cuda.synchronize()
+    return host(out, np.uint16)
+
+
+# With the workspace a last round of at most a third (a half) of the SMs'
+# tiles is split along K: (2048, 1280, 256) leaves 12 tiles for 148 SMs, two
+# pieces each (K has two blocks of 128); (2000, 1280, 384) three pieces; the
+# others take no split and must equal the plain call bit for bit.
+@pytest.mark.parametrize("mnk", [(2048, 1280, 256), (2000, 1280, 384), (64, 128, 512), (200, 300, 640)])
+def test_int8_ws_matches_oracle(mnk):
+    m, n, k = mnk
+    a_bf, w_bf = synth.w4a8_inputs(m, n, k, seed=4)
+    s2 = float(np.float32(oracle.amax_bf16(w_bf)) / np.float32(6 * 448))
+    wp, wsf = oracle.quant_nvfp4(w_bf, s2)
+    w, sw = oracle.requant_w_nvfp4_int8(wp, wsf, s2)
+    a, sa = oracle.quant_act_int8_per32(a_bf)
+    g = run_int8_ws(a, w, sa, sw)
+    ob, _, ab = oracle.int8_blockscaled_gemm(a, w, sa, sw)
+    check_tol(g, ob, ab, f"int8 ws {mnk}")
+    if mnk in ((64, 128, 512), (200, 300, 640)):
+        assert np.array_equal(g, run_int8(a, w, sa, sw))
+    assert bsq.debug_take_timeouts() == 0
+
+
+def test_int8_ws_reuse_and_determinism():
+    """Two calls on one workspace (the first leaves its counters at zero)
+    give the same bits, and a third on a fresh workspace too."""
+    m, n, k = 2000, 1280, 384
+    a_bf, w_bf = synth.w4a8_inputs(m, n, k, seed=5)
+    s2 = float(np.float32(oracle.amax_bf16(w_bf)) / np.float32(6 * 448))
+    wp, wsf = oracle.quant_nvfp4(w_bf, s2)
+    w, sw = oracle.requant_w_nvfp4_int8(wp, wsf, s2)
+    a, sa = oracle.quant_act_int8_per32(a_bf)
+    ws = torch.zeros(bsq.int8_gemm_workspace_bytes(), dtype=torch.uint8, device="cuda")
+    g1 = run_int8_ws(a, w, sa, sw, ws)
+    g2 = run_int8_ws(a, w, sa, sw, ws)
+    g3 = run_int8_ws(a, w, sa, sw)
+    assert np.array_equal(g1, g2) and np.array_equal(g1, g3)
+    assert bsq.debug_take_timeouts() == 0
+
+
 def test_int8_prefill_two_launches():
     m, n, k = 96, 256, 512
     a_bf, w_bf = synth.w4a8_inputs(m, n, k, seed=3)
