@@ -39,7 +39,9 @@
  *  - Inputs must be finite.
  *  - Concurrent calls on different streams may run concurrently; they share
  *    no device memory, except calls of int8_w4a8_prefill_noalloc, which share
- *    its scratch array and must not overlap on the GPU.
+ *    its scratch array and must not overlap on the GPU, and calls of
+ *    int8_blockscaled_gemm_ws given the same workspace, which must not
+ *    overlap either.
  *
  * Rounding: every quantised code and scale is defined bit-exactly (see each
  * function); GEMM and GEMV outputs are FP32 sums rounded once to BF16 and
