@@ -181,6 +181,17 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, FP16 x FP16 -> FP32.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // D[tmem] (+)= A * B^T, int8 x int8 -> int32 (exact).
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -332,7 +343,24 @@ __device__ __forceinline__ uint64_t sdesc_rows16(uint32_t smem_addr) {
     return d;
 }
 
+// Descriptor of a 128-row x 32-byte K-major tile without swizzle: 8 x 16 B
+// core matrices, the two along K 128 bytes apart, 8-row groups 256 bytes
+// apart (4 KB in all).
+__device__ __forceinline__ uint64_t sdesc_k_none_128x32(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+    d |= (uint64_t)(128 >> 4) << 16;    // leading byte offset: next core matrix along K
+    d |= (uint64_t)(256 >> 4) << 32;    // stride byte offset: next 8-row group
+    d |= (uint64_t)1 << 46;             // descriptor version for sm_100; layout 0 = no swizzle
+    return d;
+}
+
 // Instruction descriptors (dense, K-major A and B).
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n) {
+    return (1u << 4)                       // D = FP32
+           | (0u << 7) | (0u << 10)        // A, B = FP16 (kind::f16)
+           | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n) {
     return (1u << 4)                       // D = FP32
            | (0u << 7) | (0u << 10)        // A, B = E4M3

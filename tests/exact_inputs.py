@@ -78,3 +78,24 @@ def int8_sparse(m, n, k, seed):
     a_scale = np.where(synth.rng(seed, 924).integers(0, 2, size=(m, k // 32)) == 1, 1.0, 0.5).astype(np.float32)
     w_scale = np.where(synth.rng(seed, 925).integers(0, 2, size=(n, k // 32)) == 1, 1.0, 0.5).astype(np.float32)
     return a, w, a_scale, w_scale
+
+
+def int8_saturated(m, n, k, seed):
+    """int8 per-32 operands at the ends of the code range: each 32-block of a
+    row (of A or of W) is all -128, all 127, or a seeded mix of the two, and
+    every scale is 1.  A block's exact int32 partial then reaches +-2^19
+    (32 * 128 * 128 = 524288 for two all -128 blocks, -520192 for -128 against
+    127), the largest magnitude the format allows.  With K <= 1024 every sum
+    stays below 2^24 and is exact in FP32.  Returns (a, w, a_scale, w_scale)."""
+    assert k <= 1024 and k % 32 == 0
+
+    def side(rows, tid):
+        kind = synth.rng(seed, tid).integers(0, 3, size=(rows, k // 32))
+        mix = np.where(synth.rng(seed, tid + 1).integers(0, 2, size=(rows, k)) == 1, -128, 127)
+        kind_k = np.repeat(kind, 32, axis=1)
+        v = np.where(kind_k == 0, -128, np.where(kind_k == 1, 127, mix))
+        return v.astype(np.int8)
+
+    a = side(m, 931)
+    w = side(n, 933)
+    return a, w, np.ones((m, k // 32), np.float32), np.ones((n, k // 32), np.float32)

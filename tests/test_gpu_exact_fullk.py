@@ -15,7 +15,7 @@ import torch
 
 import int8_gemm_gemv_b200 as bsq
 import oracle
-from exact_inputs import fp8_sparse, int8_sparse, w4a4_sparse
+from exact_inputs import fp8_sparse, int8_saturated, int8_sparse, w4a4_sparse
 from gpu_helpers import bf16_out, host, to_dev
 
 
@@ -90,6 +90,29 @@ def test_int8_ws_full_k_bit_exact():
     rows = sample_rows(m, 10, 3)
     ob, _, _ = oracle.int8_blockscaled_gemm(a, w, sa, sw, rows=rows)
     _assert_bits(host(out, np.uint16)[rows], ob, "int8 ws 2048x5120x17408 exact")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mnk", [(200, 300, 640), (2048, 1280, 256), (129, 136, 1024)])
+def test_int8_saturated_blocks_bit_exact(mnk):
+    """Blocks of all -128 and all 127 codes: every block partial is as large
+    as the format allows (up to 2^19 in magnitude), through the plain call
+    and the workspace form (whose last round splits at 2048 x 1280 x 256).
+    Unit scales keep every sum exact, so the result is bit-exact."""
+    m, n, k = mnk
+    a, w, sa, sw = int8_saturated(m, n, k, seed=7)
+    ob, _, _ = oracle.int8_blockscaled_gemm(a, w, sa, sw)
+    out = bf16_out((m, n))
+    bsq.int8_blockscaled_gemm(to_dev(a), to_dev(w), to_dev(sa), to_dev(sw), out, m, n, k)
+    torch.cuda.synchronize()
+    _assert_bits(host(out, np.uint16), ob, f"int8 saturated {mnk}")
+    nbytes = bsq.int8_gemm_workspace_bytes()
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    out2 = bf16_out((m, n))
+    bsq.int8_blockscaled_gemm_ws(to_dev(a), to_dev(w), to_dev(sa), to_dev(sw), out2, ws, nbytes, m, n, k)
+    torch.cuda.synchronize()
+    _assert_bits(host(out2, np.uint16), ob, f"int8 ws saturated {mnk}")
+    assert bsq.debug_take_timeouts() == 0
 
 
 # --------------------------------------------- power of the design (CPU) ---
