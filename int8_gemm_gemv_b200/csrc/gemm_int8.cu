@@ -315,8 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         uint32_t RA[16], RB[16];  // upper / lower 16 rows of the sub-tile
         float2 acc[16];           // [row 0..3][group 0..3], a column pair each
+        // (no abort-flag read per block: if another role gives up, no more
+        // partials are committed and this bounded wait ends the fold)
         auto wait_full = [&](uint32_t g) -> bool {
-            if (!mbar_wait(&S->acc_full[g % NACC], (g / NACC) & 1, &g_timeouts) || aborted(S)) return false;
+            if (!mbar_wait(&S->acc_full[g % NACC], (g / NACC) & 1, &g_timeouts)) return false;
             tc_fence_after();
             return true;
         };
