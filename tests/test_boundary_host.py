@@ -165,3 +165,55 @@ def test_int8_ws_validation():
         bsq.BSQ_ERR_UNSUPPORTED
     assert L.int8_blockscaled_gemm_ws(A16, A16b, A16c, A16d, A16e, A16, 1 << 24, 0, 128, 128, None) == bsq.BSQ_OK
     assert bsq.debug_launch_count() == n0
+
+
+def test_int8_workspace_bytes_matches_the_device():
+    """One 64 KB piece of FP32 sums plus a 4-byte counter per SM of the
+    current device; 0 where there is no device, and the workspace call then
+    reports the CUDA failure instead of launching."""
+    torch = pytest.importorskip("torch")
+    L = bsq.lib()
+    got = bsq.int8_gemm_workspace_bytes()
+    if torch.cuda.is_available():
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        assert got == sms * (512 * 32 * 4 + 4)
+        return
+    assert got == 0
+    n0 = bsq.debug_launch_count()
+    assert L.int8_blockscaled_gemm_ws(A16, A16b, A16c, A16d, A16e, A16, 1 << 24, 128, 128, 128, None) == \
+        bsq.BSQ_ERR_CUDA
+    assert bsq.debug_launch_count() == n0
+
+
+def test_noalloc_validation():
+    """int8_w4a8_prefill_noalloc checks the shape (including the fixed
+    scratch's limit of 41,943,040 activation codes), then its pointers,
+    before any CUDA call; nothing launches."""
+    fn = bsq.lib().int8_w4a8_prefill_noalloc
+    n0 = bsq.debug_launch_count()
+    assert fn(A16, A16b, A16c, A16d, -1, 128, 128, None) == bsq.BSQ_ERR_INVALID_ARG
+    assert fn(A16, A16b, A16c, A16d, 128, 128, 48, None) == bsq.BSQ_ERR_INVALID_ARG  # K not a multiple of 32
+    assert fn(A16, A16b, A16c, A16d, 128, 128, 96, None) == bsq.BSQ_ERR_UNSUPPORTED  # nor of 128
+    assert fn(A16, A16b, A16c, A16d, 40961, 8, 1024, None) == bsq.BSQ_ERR_UNSUPPORTED  # one row past the scratch
+    # exactly at the limit the size passes, so the NULL input is what fails
+    assert fn(None, A16b, A16c, A16d, 40960, 8, 1024, None) == bsq.BSQ_ERR_INVALID_ARG
+    assert fn(A16, A16b, A16c, A16d, 0, 128, 128, None) == bsq.BSQ_OK
+    assert fn(A16, A16b, A16c, None, 128, 128, 128, None) == bsq.BSQ_ERR_INVALID_ARG
+    assert fn(ODD, A16b, A16c, A16d, 128, 128, 128, None) == bsq.BSQ_ERR_MISALIGNED
+    assert fn(A16, A16b, A16c + 4, A16d, 128, 128, 128, None) == bsq.BSQ_ERR_MISALIGNED
+    assert bsq.debug_launch_count() == n0
+
+
+def test_stream_read_validation():
+    """The plain-read probe behind the benchmark's floor rows: mode 0 or 1,
+    whole 16-byte units, a 16-byte aligned source and a 4-byte aligned sink."""
+    fn = bsq.lib().bsq_debug_stream_read
+    n0 = bsq.debug_launch_count()
+    assert fn(A16, 1024, A16b, 2, None) == bsq.BSQ_ERR_INVALID_ARG
+    assert fn(A16, 1000, A16b, 0, None) == bsq.BSQ_ERR_INVALID_ARG
+    assert fn(A16, 0, A16b, 0, None) == bsq.BSQ_OK
+    assert fn(None, 1024, A16b, 0, None) == bsq.BSQ_ERR_INVALID_ARG
+    assert fn(A16, 1024, None, 1, None) == bsq.BSQ_ERR_INVALID_ARG
+    assert fn(A16 + 8, 1024, A16b, 0, None) == bsq.BSQ_ERR_MISALIGNED
+    assert fn(A16, 1024, A16b + 2, 0, None) == bsq.BSQ_ERR_MISALIGNED
+    assert bsq.debug_launch_count() == n0
